@@ -1,0 +1,220 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) MoE-layer forward library, libmoe_b200.so.
+ *
+ * The library computes the forward pass of a top-k routed Mixture-of-Experts
+ * FFN layer with an optional always-on shared expert:
+ *
+ *     xn  = RMSNorm(h)
+ *     out = h + sum_{e in topk(score + bias)} gate_e * SwiGLU_e(xn) [+ SwiGLU_shared(xn)]
+ *
+ * as stated by the "Mixture of Experts (MoE)" lesson of AI Engineering from
+ * Scratch (Phase 07), section "The concept / Swapping the FFN" (the MoE
+ * block: scores = router(norm(h)), top_k = argmax_k(scores),
+ * h = h + sum gate(scores[e]) * Expert_e(norm(h))), with its load-balancing
+ * sections (capacity, auxiliary-loss-free bias) and "Shared experts".
+ *
+ * Conventions (every entry point):
+ *  - Every pointer argument is DEVICE memory owned by the caller, except
+ *    where a comment says "host".  The library never allocates or frees
+ *    memory and never synchronises the stream (moe_check_device_error is the
+ *    one exception, and says so).  All work is enqueued on `stream`, a
+ *    cudaStream_t passed as void* (NULL = the legacy default stream), on the
+ *    calling thread's current device.
+ *  - Tensors are dense and row-major (last index fastest), with the
+ *    element type given by moe_config.dtype ("act dtype") unless stated.
+ *    Accumulation is always fp32 or wider.
+ *  - Arguments are validated on the host before anything is launched; an
+ *    invalid call returns an error status and enqueues nothing.  Launch
+ *    failures map to MOE_ERR_CUDA.  A device-side wait that exceeds its limit
+ *    records MOE_ERR_DEVICE_TIMEOUT in the workspace header; it is reported by
+ *    moe_check_device_error.
+ *  - Calls are asynchronous: outputs are valid once the stream reaches them.
+ *    Calls that share a workspace must not overlap on the GPU.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,     /* a NULL required pointer, a bad size or a bad dtype */
+  MOE_ERR_UNSUPPORTED = 2,     /* valid, but outside what the kernels handle (e.g. bf16 d % 8 != 0) */
+  MOE_ERR_WORKSPACE = 3,       /* ws_bytes smaller than moe_workspace_size() */
+  MOE_ERR_CUDA = 4,            /* a CUDA runtime call or kernel launch failed */
+  MOE_ERR_DEVICE_TIMEOUT = 5   /* a bounded device-side wait gave up (see moe_check_device_error) */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Layer shape and options. */
+typedef struct {
+  int32_t n_tokens;        /* N >= 0 (N = 0 is a no-op) */
+  int32_t d_model;         /* d >= 1 */
+  int32_t n_experts;       /* E in [1, 1024] routed experts */
+  int32_t top_k;           /* k in [1, min(E, 32)] */
+  int32_t d_ff;            /* H >= 1, hidden width of each routed SwiGLU expert */
+  int32_t d_ff_shared;     /* Hs >= 0, hidden width of the shared expert; 0 = none */
+  int32_t dtype;           /* moe_dtype of activations and weights */
+  float rms_eps;           /* RMSNorm epsilon, >= 0 (1e-6 in every workload here) */
+  float capacity_factor;   /* <= 0: no capacity; else cap = floor(C * N * k / E) slots per expert */
+} moe_config;
+
+/* Device pointers to the layer weights (act dtype unless stated). */
+typedef struct {
+  const void* norm_w;      /* [d]          RMSNorm scale */
+  const void* w_router;    /* [E][d]       router, no bias (nn.Linear out x in) */
+  const void* w_gate;      /* [E][H][d]    routed experts, gate projection */
+  const void* w_up;        /* [E][H][d]    routed experts, up projection */
+  const void* w_down;      /* [E][d][H]    routed experts, down projection */
+  const void* ws_gate;     /* [Hs][d]      shared expert (NULL when Hs = 0) */
+  const void* ws_up;       /* [Hs][d] */
+  const void* ws_down;     /* [d][Hs] */
+} moe_weights;
+
+/* Optional device outputs of the routing steps.  Any member may be NULL; a
+ * NULL member is kept in the workspace instead (scores: not produced). */
+typedef struct {
+  float* scores;           /* [N][E]   fp32 softmax router scores */
+  int32_t* topk_idx;       /* [N][k]   chosen experts, descending score + bias, lower index first on ties */
+  float* topk_gate;        /* [N][k]   fp32 gates: chosen scores renormalised over the k */
+  int32_t* counts;         /* [E]      tokens routed to each expert before the capacity cut (sum = N*k) */
+  int32_t* offsets;        /* [E+1]    exclusive scan of the kept counts */
+  int32_t* slot_row;       /* [N*k]    row of slot t*k+j in the expert-sorted buffers, -1 = dropped */
+  int32_t* row_token;      /* [N*k]    token of each expert-sorted row (first offsets[E] valid) */
+} moe_routing;
+
+/* Optional stage timing: each non-NULL member is a cudaEvent_t recorded on
+ * the stream when moe_layer_forward reaches that point. */
+typedef struct {
+  void* start;             /* before the first kernel */
+  void* routed;            /* after RMSNorm, router, top-k (moe_route) */
+  void* permuted;          /* after counting sort and gather (moe_permute) */
+  void* gate_up;           /* after the routed gate/up + SwiGLU grouped GEMM */
+  void* down;              /* after the routed down grouped GEMM */
+  void* shared;            /* after the shared expert (== down when Hs = 0) */
+  void* combined;          /* after the combine + residual */
+} moe_trace;
+
+/* Human-readable name of a status code (static storage). */
+const char* moe_status_string(int32_t status);
+
+/* Library build string (static storage). */
+const char* moe_version(void);
+
+/* Bytes of device workspace that moe_layer_forward needs for this config,
+ * and that is also enough for every staged call below with the same config;
+ * 0 if the config is invalid.  The workspace holds a 256-byte header (device
+ * error word), xn, the routing buffers that moe_routing leaves NULL, router
+ * logits, permutation histograms, the expert-sorted rows x_perm [R][d],
+ * activations [max(R*H, N*Hs)] and expert outputs y_perm [R][d], y_shared
+ * [N][d], where R = N*k, or min(N*k, E*cap) with a capacity. */
+size_t moe_workspace_size(const moe_config* cfg);
+
+/* Zero the workspace header (the device error word).  Call once after
+ * allocating a workspace, before its first use. */
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Steps a1-a3: RMSNorm, router and top-k selection.
+ * Lesson "Step 1: the router" (scores of every expert, selection on
+ * scores + bias, gates from the chosen raw scores) and "The load-balancing
+ * problem" (DeepSeek-V3 bias on selection only).
+ *   h        [N][d]  input hidden states
+ *   norm_w   [d]     RMSNorm scale
+ *   w_router [E][d]
+ *   bias     [E]     fp32 selection bias, NULL = zeros
+ *   xn       [N][d]  out: RMSNorm(h), act dtype
+ *   scores   [N][E]  out (NULL = not written): fp32 softmax of the router logits
+ *   topk_idx [N][k], topk_gate [N][k] (fp32), counts [E]: out, as in moe_routing;
+ *                    counts is overwritten (not accumulated).
+ * xn = bf16/fp32(fl32(fl32(h * r) * w)), r = fl32(1/sqrt(mean(h^2) + eps)), mean in fp64. */
+moe_status moe_route(const moe_config* cfg, const void* h, const void* norm_w, const void* w_router,
+                     const float* bias, void* xn, float* scores, int32_t* topk_idx, float* topk_gate,
+                     int32_t* counts, void* ws, size_t ws_bytes, void* stream);
+
+/* Step a4-a5: per-expert counting sort of the N*k routing slots, capacity and
+ * gather.  Glossary "Load balancing and expert capacity" (tokens per expert,
+ * overflow continues on the residual); lesson "The load-balancing problem"
+ * (capacity C x N / E); "Expert parallelism for MoE serving", "Technical
+ * insight" (dispatch groups tokens by expert; capacity keeps GEMM shapes
+ * predictable).  Slot s = t*k + j is ranked among the slots of its expert
+ * in increasing s; ranks >= cap are dropped (slot_row = -1).
+ *   topk_idx  [N][k] in
+ *   xn        [N][d] in
+ *   offsets   [E+1]  out: offsets[e] = sum of kept counts of experts < e
+ *   slot_row  [N*k]  out
+ *   row_token [N*k]  out (first offsets[E] entries valid)
+ *   x_perm    [R][d] out: x_perm[slot_row[s]] = xn[s / k] for kept slots */
+moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* xn, int32_t* offsets,
+                       int32_t* slot_row, int32_t* row_token, void* x_perm, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* Steps a6-a8: grouped SwiGLU expert FFN, y = W_down(silu(W_gate x) * (W_up x)).
+ * Lesson "The concept" (each expert an independent FFN, usually SwiGLU);
+ * "Expert parallelism for MoE serving", "Future" (GEMM units that batch many
+ * experts).  Rows [offsets[g], offsets[g+1]) of x use expert g's weights.
+ *   n_groups  G >= 1 experts stacked in w_gate/w_up [G][d_ff][d], w_down [G][d][d_ff]
+ *   offsets   [G+1] device, nondecreasing, offsets[G] <= max_rows; NULL = one
+ *             group of max_rows rows (the shared expert: x = xn, max_rows = N)
+ *   max_rows  rows that x and y hold (a host-side bound on offsets[G])
+ *   x         [max_rows][d] in;  y [max_rows][d] out, act dtype; rows at or
+ *             past offsets[G] are not written.
+ * The SwiGLU activation (act dtype) is kept in the workspace. */
+moe_status moe_expert_ffn(const moe_config* cfg, int32_t n_groups, const int32_t* offsets, int32_t max_rows,
+                          const void* x, const void* w_gate, const void* w_up, const void* w_down,
+                          int32_t d_ff, void* y, void* ws, size_t ws_bytes, void* stream);
+
+/* Step a9: gated combine plus residual, in gather form (deterministic):
+ * out[t] = h[t] + sum_{j, slot kept} gate[t][j] * y_perm[slot_row[t*k+j]] (+ y_shared[t]),
+ * summed in fp32 and rounded once.  Lesson MoE block (h + sum gate * Expert);
+ * glossary example (out[token] += weight * expert(token)).
+ *   h [N][d], y_perm [R][d], slot_row [N*k], topk_gate [N][k] fp32,
+ *   y_shared [N][d] or NULL, out [N][d] (may equal h). */
+moe_status moe_combine(const moe_config* cfg, const void* h, const void* y_perm, const int32_t* slot_row,
+                       const float* topk_gate, const void* y_shared, void* out, void* stream);
+
+/* The whole forward pass: moe_route, moe_permute, moe_expert_ffn (routed
+ * experts, then the shared expert when Hs > 0) and moe_combine, on one
+ * stream with no host synchronisation.
+ *   weights   device pointers (struct itself on the host)
+ *   h [N][d] in, bias [E] fp32 or NULL, out [N][d] (may equal h)
+ *   routing   host struct of optional device outputs, or NULL
+ *   trace     host struct of optional cudaEvent_t, or NULL */
+moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* weights, const void* h,
+                             const float* bias, void* out, const moe_routing* routing,
+                             const moe_trace* trace, void* ws, size_t ws_bytes, void* stream);
+
+/* Step a10: auxiliary-loss-free bias update.  Lesson "The load-balancing
+ * problem" (after each step, +-gamma per expert by usage above or below
+ * target) and "Step 2" (-gamma for over-used, +gamma for under-used experts):
+ *   bias[e] = fl32(bias[e] + gamma * sign(target - counts[e])), sign(0) = 0.
+ *   counts [E] int32 in, bias [E] fp32 in/out. */
+moe_status moe_bias_update(int32_t n_experts, const int32_t* counts, float target, float gamma, float* bias,
+                           void* stream);
+
+/* Synchronise `stream`, read and clear the workspace's device error word.
+ * Returns MOE_OK, the recorded status (e.g. MOE_ERR_DEVICE_TIMEOUT) or
+ * MOE_ERR_CUDA.  info (host, may be NULL) receives 4 int32 of detail
+ * (status, kernel id, block, wait site).  This call blocks the host. */
+moe_status moe_check_device_error(void* ws, size_t ws_bytes, void* stream, int32_t* info);
+
+/* Limit, in nanoseconds, of every bounded device-side wait in kernels
+ * launched after this call (process-wide; default 2e9 = 2 s; 0 = give up at
+ * the first unsuccessful poll). */
+moe_status moe_set_wait_timeout_ns(int64_t ns);
+
+/* Launch one block that waits on a workspace flag that nothing sets, with
+ * the current wait limit: it must give up and record MOE_ERR_DEVICE_TIMEOUT.
+ * Exercises the timeout path without faulting or hanging the GPU. */
+moe_status moe_selftest_wait_timeout(void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,130 @@
+// Steps a9 and a10 of the MoE layer: the gated combine fused with the
+// residual add, and the auxiliary-loss-free bias update.
+//
+// Sources: "Mixture of Experts (MoE)" lesson (AI Engineering from Scratch,
+// Phase 07), "The concept / Swapping the FFN" (h = h + sum over the chosen
+// experts of gate * Expert(norm(h))), "Shared experts" (every token also
+// passes the shared expert), "The load-balancing problem" and "Step 2"
+// (after each step every expert's bias moves by -gamma when it was used above
+// the target and by +gamma when below); Ultralytics glossary "Mixture of
+// Experts (MoE)" example (out[token] += weight * expert(token)) and "Load
+// balancing and expert capacity" (a dropped token continues on the residual).
+#include "moe_common.cuh"
+#include "moe_kernels.h"
+
+namespace moe {
+
+// Gather form: each output element reads its token's k expert rows, so no
+// atomics are needed and the sum order is fixed:
+//   acc = h; acc = fma(gate_j, y_j, acc) for kept j in rank order; acc += y_shared;
+//   out = round(acc).
+// A token whose slots are all dropped (and no shared expert) returns h exactly.
+// VEC consecutive elements per thread (VEC * sizeof(T) = 16 bytes when aligned).
+template <typename T, int VEC>
+__global__ void __launch_bounds__(128) combine_kernel(const T* __restrict__ h, const T* __restrict__ y_perm,
+                                                      const int32_t* __restrict__ slot_row,
+                                                      const float* __restrict__ gates,
+                                                      const T* __restrict__ y_shared, T* out, int n, int d,
+                                                      int k) {
+  __shared__ int32_t rows[32];
+  __shared__ float g[32];
+  for (int t = blockIdx.x; t < n; t += gridDim.x) {
+    if (threadIdx.x < k) {
+      rows[threadIdx.x] = slot_row[(size_t)t * k + threadIdx.x];
+      g[threadIdx.x] = gates[(size_t)t * k + threadIdx.x];
+    }
+    __syncthreads();
+    for (int c = threadIdx.x * VEC; c < d; c += blockDim.x * VEC) {
+      float acc[VEC];
+      T tmp[VEC];
+      const size_t off = (size_t)t * d + c;
+      if (VEC > 1) {
+        *reinterpret_cast<uint4*>(tmp) = *reinterpret_cast<const uint4*>(h + off);
+      } else {
+        tmp[0] = h[off];
+      }
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) acc[i] = to_f32(tmp[i]);
+      for (int j = 0; j < k; ++j) {
+        const int r = rows[j];
+        if (r < 0) continue;
+        const float gj = g[j];
+        const T* yr = y_perm + (size_t)r * d + c;
+        if (VEC > 1) {
+          *reinterpret_cast<uint4*>(tmp) = *reinterpret_cast<const uint4*>(yr);
+        } else {
+          tmp[0] = yr[0];
+        }
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) acc[i] = __fmaf_rn(gj, to_f32(tmp[i]), acc[i]);
+      }
+      if (y_shared != nullptr) {
+        if (VEC > 1) {
+          *reinterpret_cast<uint4*>(tmp) = *reinterpret_cast<const uint4*>(y_shared + off);
+        } else {
+          tmp[0] = y_shared[off];
+        }
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) acc[i] = __fadd_rn(acc[i], to_f32(tmp[i]));
+      }
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) tmp[i] = from_f32<T>(acc[i]);
+      if (VEC > 1) {
+        *reinterpret_cast<uint4*>(out + off) = *reinterpret_cast<const uint4*>(tmp);
+      } else {
+        out[off] = tmp[0];
+      }
+    }
+    __syncthreads();
+  }
+}
+
+// bias[e] = fl32(bias[e] + gamma * s), s = sign(target - counts[e]) in {-1, 0, +1}.
+__global__ void bias_update_kernel(int E, const int32_t* __restrict__ counts, float target, float gamma,
+                                   float* __restrict__ bias) {
+  int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= E) return;
+  float c = (float)counts[e];
+  float s = (target > c) ? 1.f : ((target < c) ? -1.f : 0.f);
+  bias[e] = __fadd_rn(bias[e], __fmul_rn(s, gamma));
+}
+
+}  // namespace moe
+
+namespace moe_host {
+
+moe_status launch_combine(int dtype, const void* h, const void* y_perm, const int32_t* slot_row,
+                          const float* topk_gate, const void* y_shared, void* out, int n, int d, int k,
+                          cudaStream_t s) {
+  if (n == 0) return MOE_OK;
+  int grid = n < sm_count() * 16 ? n : sm_count() * 16;
+  const uintptr_t addr = (uintptr_t)h | (uintptr_t)y_perm | (uintptr_t)y_shared | (uintptr_t)out;
+  if (dtype == MOE_BF16) {
+    typedef moe::bf16 T;
+    if (d % 8 == 0 && addr % 16 == 0)
+      moe::combine_kernel<T, 8><<<grid, 128, 0, s>>>((const T*)h, (const T*)y_perm, slot_row, topk_gate,
+                                                     (const T*)y_shared, (T*)out, n, d, k);
+    else
+      moe::combine_kernel<T, 1><<<grid, 128, 0, s>>>((const T*)h, (const T*)y_perm, slot_row, topk_gate,
+                                                     (const T*)y_shared, (T*)out, n, d, k);
+  } else {
+    if (d % 4 == 0 && addr % 16 == 0)
+      moe::combine_kernel<float, 4><<<grid, 128, 0, s>>>((const float*)h, (const float*)y_perm, slot_row,
+                                                         topk_gate, (const float*)y_shared, (float*)out, n, d,
+                                                         k);
+    else
+      moe::combine_kernel<float, 1><<<grid, 128, 0, s>>>((const float*)h, (const float*)y_perm, slot_row,
+                                                         topk_gate, (const float*)y_shared, (float*)out, n, d,
+                                                         k);
+  }
+  return launch_status();
+}
+
+moe_status launch_bias_update(int e, const int32_t* counts, float target, float gamma, float* bias,
+                              cudaStream_t s) {
+  if (e == 0) return MOE_OK;
+  moe::bias_update_kernel<<<(e + 255) / 256, 256, 0, s>>>(e, counts, target, gamma, bias);
+  return launch_status();
+}
+
+}  // namespace moe_host

@@ -1,0 +1,64 @@
+// Host-side launchers of the library's kernels.  Each enqueues work on
+// `stream` and returns cudaGetLastError() mapped to a moe_status; none
+// allocates or synchronises.  Argument checking happens in moe_api.cu.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe_host {
+
+// a1: xn = RMSNorm(h) (one block per token).
+moe_status launch_rmsnorm(int dtype, const void* h, const void* norm_w, void* xn, int n, int d, float eps,
+                          cudaStream_t s);
+
+// a3: softmax over the router logits, top-k on score + bias, renormalised
+// gates and the per-expert counts (counts are zeroed here first).
+moe_status launch_topk(const float* logits, const float* bias, float* scores, int32_t* topk_idx,
+                       float* topk_gate, int32_t* counts, int n, int e, int k, cudaStream_t s);
+
+// a4: stable counting sort of the N*k slots by expert with optional capacity.
+//   hist: workspace of permute_hist_ints(n*k, e) int32.
+size_t permute_hist_ints(int64_t slots, int e);
+moe_status launch_permute(const int32_t* topk_idx, int n, int k, int e, int cap, int32_t* hist,
+                          int32_t* offsets, int32_t* slot_row, int32_t* row_token, cudaStream_t s);
+
+// a5: x_perm[r] = xn[row_token[r]] for r < offsets[e] (device count).
+moe_status launch_gather(int dtype, const void* xn, const int32_t* row_token, const int32_t* offsets, int e,
+                         void* x_perm, int max_rows, int d, cudaStream_t s);
+
+// a9: out = h + sum_j gate_j * y_perm[slot_row] (+ y_shared).
+moe_status launch_combine(int dtype, const void* h, const void* y_perm, const int32_t* slot_row,
+                          const float* topk_gate, const void* y_shared, void* out, int n, int d, int k,
+                          cudaStream_t s);
+
+// a10: bias[e] += gamma * sign(target - counts[e]).
+moe_status launch_bias_update(int e, const int32_t* counts, float target, float gamma, float* bias,
+                              cudaStream_t s);
+
+// Grouped GEMM epilogues.
+enum GemmEpilogue { EPI_F32 = 0, EPI_SWIGLU = 1, EPI_STORE = 2 };
+
+// Grouped GEMM on CUDA cores (fp32 or bf16 operands, fp32 accumulation):
+//   rows [off[g], off[g+1]) of A [max_rows][k] times B_g^T, B_g = B + g*nout*k ([nout][k]).
+//   EPI_SWIGLU: C = silu(A B_g^T) * (A B2_g^T) in the act dtype;
+//   EPI_STORE: C = A B_g^T in the act dtype; EPI_F32: C = A B_g^T in fp32.
+//   offsets == nullptr: one group of max_rows rows.  ldc = row stride of C.
+moe_status launch_gemm_simt(int dtype, int epi, const void* a, const void* b, const void* b2,
+                            const int32_t* offsets, int groups, int max_rows, int nout, int k, void* c,
+                            int ldc, cudaStream_t s);
+
+// The same grouped GEMM on the tcgen05 tensor cores (bf16 operands only,
+// TMA-fed, TMEM accumulators, persistent over the SMs).  k % 8 == 0.
+//   hdr: workspace header that receives a device time-out, if any.
+moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2, const int32_t* offsets,
+                          int groups, int max_rows, int nout, int k, void* c, int ldc, int32_t* hdr,
+                          cudaStream_t s);
+
+// A block that waits, with the bounded wait of the pipelined kernels, on a
+// barrier that nothing completes.
+moe_status launch_selftest_wait(int32_t* hdr, cudaStream_t s);
+
+}  // namespace moe_host

@@ -1,0 +1,223 @@
+// Steps a4 and a5 of the MoE layer: per-expert counting sort of the N*k
+// routing slots with an optional capacity, and the gather of token rows into
+// expert-contiguous buffers.
+//
+// Sources: Ultralytics glossary "Mixture of Experts (MoE)", "Load balancing
+// and expert capacity" (tokens per expert; tokens over an expert's limit
+// continue on the residual) and its top-2 example (each expert takes the
+// tokens that chose it, in token order); "Mixture of Experts (MoE)" lesson,
+// "The load-balancing problem" (expert capacity C x N / E, overflow tokens
+// pass the layer); "Expert parallelism for MoE serving", "Technical insight"
+// (dispatch groups each expert's tokens; capacity keeps GEMM shapes
+// predictable).
+//
+// Slot s = t*k + j.  Its rank within expert e is the number of slots s' < s
+// routed to e; with a capacity, ranks >= cap are dropped.  The order is fixed
+// by the slot index alone (no atomics decide it), so the result is
+// deterministic and equals a stable sort.
+//
+// Kernels: (1) one warp per chunk of 256 slots counts the chunk's slots per
+// expert into hist[e][chunk]; (2) one block scans hist in expert-major order
+// (giving every chunk its starting position within its expert) and forms the
+// kept counts and offsets; (3) the chunk warps recompute their in-chunk ranks
+// and write slot_row / row_token; (4) the gather copies rows with 16-byte
+// loads.
+#include "moe_common.cuh"
+#include "moe_kernels.h"
+
+namespace moe {
+
+constexpr int kChunk = 256;        // slots per warp
+constexpr int kPermWarps = 4;      // warps per block in kernels (1) and (3)
+
+// In-chunk ranking shared by kernels (1) and (3).  `run` is this warp's
+// shared running count per expert (zeroed by the caller).  For each slot of
+// the chunk in increasing order, calls f(slot, expert, rank_in_chunk).
+template <typename F>
+__device__ __forceinline__ void chunk_walk(const int32_t* __restrict__ idx, int64_t slots, int64_t c,
+                                           int32_t* run, F f) {
+  const int lane = lane_id();
+  const unsigned lt = (1u << lane) - 1u;
+  for (int step = 0; step < kChunk / 32; ++step) {
+    int64_t s = c * kChunk + step * 32 + lane;
+    int e = (s < slots) ? idx[s] : -1;
+    unsigned same = __match_any_sync(0xffffffffu, e);
+    int before = __popc(same & lt);
+    int base = (e >= 0) ? run[e] : 0;
+    __syncwarp();
+    if (e >= 0) {
+      f(s, e, base + before);
+      if (before == 0) run[e] = base + __popc(same);  // the lowest lane of each group
+    }
+    __syncwarp();
+  }
+}
+
+__global__ void __launch_bounds__(kPermWarps * 32) chunk_hist_kernel(const int32_t* __restrict__ idx,
+                                                                     int64_t slots, int E, int nchunks,
+                                                                     int32_t* __restrict__ hist) {
+  extern __shared__ int32_t run_all[];
+  int32_t* run = run_all + warp_id() * E;
+  int64_t c = (int64_t)blockIdx.x * kPermWarps + warp_id();
+  for (int e = lane_id(); e < E; e += 32) run[e] = 0;
+  __syncwarp();
+  if (c >= nchunks) return;
+  chunk_walk(idx, slots, c, run, [](int64_t, int, int) {});
+  for (int e = lane_id(); e < E; e += 32) hist[(int64_t)e * nchunks + c] = run[e];
+}
+
+// One block of 1024 threads.  Exclusive scan of hist (E*nchunks ints,
+// expert-major) in place, tile by tile with a running carry; then
+//   count_e = start_{e+1} - start_e, kept_e = min(count_e, cap),
+//   offsets = exclusive scan of kept (E+1 entries).
+__global__ void __launch_bounds__(1024) hist_scan_kernel(int32_t* __restrict__ hist, int64_t len, int E,
+                                                         int nchunks, int64_t slots, int cap,
+                                                         int32_t* __restrict__ offsets) {
+  constexpr int PER = 8;
+  __shared__ int32_t warp_sum[32];
+  __shared__ int32_t carry_sh;
+  __shared__ int32_t kept_sh[1024];
+  const int tid = threadIdx.x;
+  if (tid == 0) carry_sh = 0;
+  __syncthreads();
+  for (int64_t base = 0; base < len; base += 1024 * PER) {
+    int32_t v[PER];
+    int32_t local = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      int64_t p = base + (int64_t)tid * PER + i;
+      v[i] = (p < len) ? hist[p] : 0;
+      local += v[i];
+    }
+    // block-wide exclusive scan of `local`
+    int32_t x = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane_id() >= o) x += y;
+    }
+    if (lane_id() == 31) warp_sum[warp_id()] = x;
+    __syncthreads();
+    if (warp_id() == 0) {
+      int32_t w = warp_sum[lane_id()];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane_id() >= o) w += y;
+      }
+      warp_sum[lane_id()] = w;  // inclusive
+    }
+    __syncthreads();
+    int32_t carry = carry_sh;
+    int32_t excl = carry + (x - local) + (warp_id() > 0 ? warp_sum[warp_id() - 1] : 0);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      int64_t p = base + (int64_t)tid * PER + i;
+      if (p < len) hist[p] = excl;
+      excl += v[i];
+    }
+    __syncthreads();
+    if (tid == 0) carry_sh = carry + warp_sum[31];
+    __syncthreads();
+  }
+  // kept counts and their exclusive scan (E <= 1024: one expert per thread)
+  int32_t kept = 0;
+  if (tid < E) {
+    int32_t start = hist[(int64_t)tid * nchunks];
+    int32_t end = (tid + 1 < E) ? hist[(int64_t)(tid + 1) * nchunks] : (int32_t)slots;
+    kept = end - start;
+    if (cap >= 0 && kept > cap) kept = cap;
+  }
+  kept_sh[tid] = kept;
+  __syncthreads();
+  if (tid == 0) {
+    int32_t acc = 0;
+    for (int e = 0; e < E; ++e) {
+      offsets[e] = acc;
+      acc += kept_sh[e];
+    }
+    offsets[E] = acc;
+  }
+}
+
+__global__ void __launch_bounds__(kPermWarps * 32) chunk_scatter_kernel(
+    const int32_t* __restrict__ idx, int64_t slots, int k, int E, int nchunks, int cap,
+    const int32_t* __restrict__ hist, const int32_t* __restrict__ offsets, int32_t* __restrict__ slot_row,
+    int32_t* __restrict__ row_token) {
+  extern __shared__ int32_t run_all[];
+  int32_t* run = run_all + warp_id() * E;
+  int64_t c = (int64_t)blockIdx.x * kPermWarps + warp_id();
+  for (int e = lane_id(); e < E; e += 32) run[e] = 0;
+  __syncwarp();
+  if (c >= nchunks) return;
+  chunk_walk(idx, slots, c, run, [&](int64_t s, int e, int r_in_chunk) {
+    int32_t rank = hist[(int64_t)e * nchunks + c] - hist[(int64_t)e * nchunks] + r_in_chunk;
+    if (cap < 0 || rank < cap) {
+      int32_t row = offsets[e] + rank;
+      slot_row[s] = row;
+      row_token[row] = (int32_t)(s / k);
+    } else {
+      slot_row[s] = -1;
+    }
+  });
+}
+
+// a5: x_perm[r] = xn[row_token[r]] for r < offsets[E].  One block per row,
+// grid-stride; VEC elements per 16-byte access when the row allows it.
+template <typename V>
+__global__ void __launch_bounds__(128) gather_rows_kernel(const V* __restrict__ xn,
+                                                          const int32_t* __restrict__ row_token,
+                                                          const int32_t* __restrict__ offsets, int E,
+                                                          V* __restrict__ x_perm, int row_vecs) {
+  const int rows = offsets[E];
+  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+    const V* src = xn + (size_t)row_token[r] * row_vecs;
+    V* dst = x_perm + (size_t)r * row_vecs;
+    for (int i = threadIdx.x; i < row_vecs; i += blockDim.x) dst[i] = src[i];
+  }
+}
+
+}  // namespace moe
+
+namespace moe_host {
+
+static inline int64_t n_chunks(int64_t slots) { return (slots + moe::kChunk - 1) / moe::kChunk; }
+
+size_t permute_hist_ints(int64_t slots, int e) { return (size_t)(n_chunks(slots) > 0 ? n_chunks(slots) : 1) * e; }
+
+moe_status launch_permute(const int32_t* topk_idx, int n, int k, int e, int cap, int32_t* hist,
+                          int32_t* offsets, int32_t* slot_row, int32_t* row_token, cudaStream_t s) {
+  const int64_t slots = (int64_t)n * k;
+  const int64_t nch = n_chunks(slots);
+  if (nch == 0) {
+    if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (e + 1), s) != cudaSuccess) return MOE_ERR_CUDA;
+    return MOE_OK;
+  }
+  const int blocks = (int)((nch + moe::kPermWarps - 1) / moe::kPermWarps);
+  const size_t smem = sizeof(int32_t) * e * moe::kPermWarps;
+  moe::chunk_hist_kernel<<<blocks, moe::kPermWarps * 32, smem, s>>>(topk_idx, slots, e, (int)nch, hist);
+  moe::hist_scan_kernel<<<1, 1024, 0, s>>>(hist, nch * e, e, (int)nch, slots, cap, offsets);
+  moe::chunk_scatter_kernel<<<blocks, moe::kPermWarps * 32, smem, s>>>(topk_idx, slots, k, e, (int)nch, cap,
+                                                                       hist, offsets, slot_row, row_token);
+  return launch_status();
+}
+
+moe_status launch_gather(int dtype, const void* xn, const int32_t* row_token, const int32_t* offsets, int e,
+                         void* x_perm, int max_rows, int d, cudaStream_t s) {
+  if (max_rows == 0) return MOE_OK;
+  const size_t row_bytes = (size_t)d * (dtype == MOE_BF16 ? 2 : 4);
+  int grid = max_rows < sm_count() * 16 ? max_rows : sm_count() * 16;
+  const uintptr_t addr = (uintptr_t)xn | (uintptr_t)x_perm;
+  if (row_bytes % 16 == 0 && addr % 16 == 0)
+    moe::gather_rows_kernel<uint4><<<grid, 128, 0, s>>>((const uint4*)xn, row_token, offsets, e, (uint4*)x_perm,
+                                                        (int)(row_bytes / 16));
+  else if (row_bytes % 4 == 0 && addr % 4 == 0)
+    moe::gather_rows_kernel<uint32_t><<<grid, 128, 0, s>>>((const uint32_t*)xn, row_token, offsets, e,
+                                                           (uint32_t*)x_perm, (int)(row_bytes / 4));
+  else
+    moe::gather_rows_kernel<uint16_t><<<grid, 128, 0, s>>>((const uint16_t*)xn, row_token, offsets, e,
+                                                           (uint16_t*)x_perm, (int)(row_bytes / 2));
+  return launch_status();
+}
+
+}  // namespace moe_host

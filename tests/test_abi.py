@@ -1,0 +1,99 @@
+"""The C ABI without a GPU: the library loads, exports every entry point that
+include/moe.h declares, sizes workspaces and rejects bad arguments on the
+host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_mixture_experts_rmsnorm_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    declared = _declared_functions()
+    assert len(declared) >= 13
+    lib = ctypes.CDLL(moe.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert sorted(moe.ENTRY_POINTS) == declared
+
+
+def test_status_strings_and_version():
+    lib = moe.library()
+    for st in range(6):
+        assert lib.moe_status_string(st).decode().startswith("MOE_")
+    assert "sm_100a" in moe.version()
+
+
+def _cfg(**kw):
+    base = dict(n_tokens=256, d_model=64, n_experts=8, top_k=2, d_ff=128, dtype="f32")
+    base.update(kw)
+    return moe.Config(**base)
+
+
+def test_workspace_size_grows_with_shape_and_rejects_bad_configs():
+    a = moe.workspace_size(_cfg())
+    assert a > 0 and a % 256 == 0
+    assert moe.workspace_size(_cfg(n_tokens=512)) > a
+    assert moe.workspace_size(_cfg(d_ff_shared=64)) > a
+    # capacity shrinks the expert-sorted buffers
+    assert moe.workspace_size(_cfg(capacity_factor=0.5)) < a
+    for bad in (dict(top_k=9), dict(top_k=0), dict(n_experts=0), dict(n_experts=2000, top_k=2),
+                dict(d_model=0), dict(n_tokens=-1), dict(d_ff=0), dict(top_k=33, n_experts=64)):
+        assert moe.workspace_size(_cfg(**bad)) == 0, bad
+
+
+def test_workspace_bytes_match_the_documented_regions():
+    c = _cfg(dtype="bf16", n_tokens=1000, d_model=512, n_experts=16, top_k=4, d_ff=384, d_ff_shared=256)
+    R = c.rows
+    es = 2
+    need = (c.n_tokens * c.d_model * es + c.n_tokens * c.n_experts * 4 + 4 * c.n_tokens * c.top_k * 4
+            + R * c.d_model * es * 2 + max(R * c.d_ff, c.n_tokens * c.d_ff_shared) * es
+            + c.n_tokens * c.d_model * es)
+    got = moe.workspace_size(c)
+    assert need <= got <= need + 64 * 1024
+
+
+def test_host_validation_before_any_launch():
+    lib = moe.library()
+    bad = _cfg(top_k=9).c()
+    st = lib.moe_route(ctypes.byref(bad), None, None, None, None, None, None, None, None, None, None, 0, None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+    good = _cfg().c()
+    # a workspace pointer that is not 256-byte aligned
+    st = lib.moe_route(ctypes.byref(good), 16, 16, 16, None, 16, None, 16, 16, 16, 16 + 8, 1 << 30, None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+    # a workspace smaller than moe_workspace_size
+    st = lib.moe_route(ctypes.byref(good), 256, 256, 256, None, 256, None, 256, 256, 256, 256, 1024, None)
+    assert st == moe.MOE_ERR_WORKSPACE
+    # bf16 rows that are not whole 16-byte units
+    odd = _cfg(dtype="bf16", d_model=60).c()
+    st = lib.moe_permute(ctypes.byref(odd), 256, 256, 256, 256, 256, 256, 256, 1 << 30, None)
+    assert st == moe.MOE_ERR_UNSUPPORTED
+    # expert FFN: group count and act capacity
+    st = lib.moe_expert_ffn(ctypes.byref(good), 0, None, 16, 256, 256, 256, 256, 128, 256, 256, 1 << 30, None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+    st = lib.moe_expert_ffn(ctypes.byref(good), 2, None, 16, 256, 256, 256, 256, 128, 256, 256, 1 << 30, None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+    st = lib.moe_expert_ffn(ctypes.byref(good), 1, None, 100000, 256, 256, 256, 256, 128, 256, 256, 1 << 30, None)
+    assert st == moe.MOE_ERR_WORKSPACE
+    assert lib.moe_bias_update(0, 256, 1.0, 1e-3, 256, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_set_wait_timeout_ns(-1) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_check_device_error(None, 0, None, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_python_wrapper_raises_on_error_status():
+    with pytest.raises(moe.MoEError) as ei:
+        moe.moe_set_wait_timeout_ns(-5)
+    assert ei.value.status == moe.MOE_ERR_INVALID_ARG
+    moe.moe_set_wait_timeout_ns(2_000_000_000)

@@ -1,0 +1,264 @@
+"""GPU parity of the MoE-layer forward against the CPU oracle, through the C ABI.
+
+Every test here needs a B200 (sm_100a).  Routing, counts, permutation and
+drop masks are compared bit-exactly (tokens whose oracle selection keys are
+within 1e-6 of each other are skipped); outputs within max-abs 1e-4 (fp32
+layer) or 2e-2 of the output RMS (bf16 layers, fp32 accumulation); bias
+updates bit-exactly.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import moe_inputs as mi
+import oracle
+from parity_helpers import (BF16_REL_RMS, F32_MAX_ABS, check_permutation, check_routing, lib_config,
+                            oracle_outputs, oracle_routing, rel_rms_err, run_gpu_layer, to_np)
+
+pytestmark = pytest.mark.gpu
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(scope="module")
+def torch_cuda():
+    import torch
+    assert torch.cuda.is_available()
+    import sparse_mixture_experts_rmsnorm_b200  # noqa: F401  (fails loudly when the library is missing)
+    if not os.path.exists(mi.CUDA_LIB):
+        mi.build(cuda=True)
+    return torch
+
+
+def _full_oracle(cfg):
+    a = {n: mi.host_tensor(cfg, n) for n in mi.layer_tensor_specs(cfg)}
+    return oracle.layer_forward(a["h"], a["norm_w"], a["w_router"], a["bias"], a["w_gate"], a["w_up"],
+                                a["w_down"], top_k=cfg.top_k, eps=cfg.rms_eps, dtype=cfg.dtype,
+                                capacity_factor=cfg.capacity_factor, ws_gate=a.get("ws_gate"),
+                                ws_up=a.get("ws_up"), ws_down=a.get("ws_down"))
+
+
+# ----------------------------------------------------------------- generator
+
+def test_device_generator_matches_host(torch_cuda):
+    cfg = mi.CONFIGS["dsv3_decode_bf16"]
+    dev = mi.device_tensors(cfg, names=["h", "bias", "w_router"])
+    for n in ("h", "bias", "w_router"):
+        np.testing.assert_array_equal(to_np(dev[n]).astype(np.float32), mi.host_tensor(cfg, n))
+
+
+# ----------------------------------------------------------------- tiny fp32, whole layer
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_tiny_fp32_layer_matches_oracle(torch_cuda, seed):
+    cfg = mi.CONFIGS["tiny_fp32"].with_(seed=seed)
+    g = run_gpu_layer(cfg)
+    ref = _full_oracle(cfg)
+    np.testing.assert_array_equal(g["xn"], ref["xn"])
+    skipped = check_routing(g, {"key": ref["key"], "idx": ref["idx"], "gates": ref["gates"],
+                                "scores": ref["scores"]}, cfg.top_k)
+    assert skipped == 0
+    check_permutation(g, cfg.n_experts, -1)
+    err = np.max(np.abs(g["out"] - ref["out64"]))
+    assert err <= F32_MAX_ABS, err
+
+
+def test_tiny_fp32_staged_calls_equal_layer_forward(torch_cuda):
+    torch = torch_cuda
+    import sparse_mixture_experts_rmsnorm_b200 as moe
+    cfg = mi.CONFIGS["tiny_fp32"]
+    lc = lib_config(cfg)
+    dev = mi.device_tensors(cfg)
+    g = run_gpu_layer(cfg, dev=dev)
+    N, d, E, k, H = cfg.n_tokens, cfg.d_model, cfg.n_experts, cfg.top_k, cfg.d_ff
+    ws = moe.workspace(lc)
+    kw = dict(device="cuda")
+    xn = torch.empty(N, d, **kw)
+    idx = torch.empty(N, k, dtype=torch.int32, **kw)
+    gate = torch.empty(N, k, **kw)
+    counts = torch.empty(E, dtype=torch.int32, **kw)
+    moe.moe_route(lc, dev["h"], dev["norm_w"], dev["w_router"], None, xn, None, idx, gate, counts, ws)
+    offsets = torch.empty(E + 1, dtype=torch.int32, **kw)
+    slot_row = torch.empty(N * k, dtype=torch.int32, **kw)
+    row_token = torch.empty(N * k, dtype=torch.int32, **kw)
+    x_perm = torch.empty(N * k, d, **kw)
+    moe.moe_permute(lc, idx, xn, offsets, slot_row, row_token, x_perm, ws)
+    y = torch.full((N * k, d), float("nan"), **kw)
+    moe.moe_expert_ffn(lc, E, offsets, N * k, x_perm, dev["w_gate"], dev["w_up"], dev["w_down"], H, y, ws)
+    out = torch.empty(N, d, **kw)
+    moe.moe_combine(lc, dev["h"], y, slot_row, gate, None, out, None)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(to_np(idx), g["topk_idx"])
+    np.testing.assert_array_equal(to_np(slot_row), g["slot_row"])
+    np.testing.assert_array_equal(to_np(out), g["out"])
+    # x_perm rows are the tokens' xn rows
+    np.testing.assert_array_equal(to_np(x_perm), to_np(xn)[g["row_token"]])
+
+
+def test_single_expert_and_dense_identities(torch_cuda):
+    # E = 1, k = 1: the textbook SwiGLU FFN; k = E (zero bias): dense softmax-weighted sum.
+    for over in (dict(n_experts=1, top_k=1), dict(n_experts=4, top_k=4), dict(n_experts=8, top_k=8)):
+        cfg = mi.CONFIGS["tiny_fp32"].with_(**over)
+        g = run_gpu_layer(cfg)
+        ref = _full_oracle(cfg)
+        assert np.all(g["counts"] == cfg.n_tokens)
+        err = np.max(np.abs(g["out"] - ref["out64"]))
+        assert err <= F32_MAX_ABS, (over, err)
+
+
+def test_exact_ties_choose_lower_expert_index(torch_cuda):
+    torch = torch_cuda
+    cfg = mi.CONFIGS["tiny_fp32"].with_(n_tokens=64)
+    dev = mi.device_tensors(cfg)
+    dev["w_router"].zero_()  # every logit 0: all scores equal
+    g = run_gpu_layer(cfg, dev=dev)
+    assert np.all(g["topk_idx"] == np.array([[0, 1]]))
+    np.testing.assert_array_equal(g["topk_gate"], 0.5)
+    # a bias breaks the tie in favour of experts 5 and 2
+    dev["bias"].copy_(torch.tensor([0, 0, 1e-3, 0, 0, 2e-3, 0, 0], dtype=torch.float32))
+    g = run_gpu_layer(cfg, dev=dev)
+    assert np.all(g["topk_idx"] == np.array([[5, 2]]))
+    np.testing.assert_array_equal(g["topk_gate"], 0.5)
+
+
+def test_empty_input_is_a_no_op(torch_cuda):
+    cfg = mi.CONFIGS["tiny_fp32"].with_(n_tokens=0)
+    g = run_gpu_layer(cfg)
+    assert g["out"].shape == (0, cfg.d_model)
+    assert np.all(g["counts"] == 0) and np.all(g["offsets"] == 0)
+
+
+# ----------------------------------------------------------------- permutation on the printed example
+
+@pytest.mark.parametrize("capacity_factor,expect_offsets", [
+    (0.0, [0, 1, 3, 4, 7, 7, 7, 10, 12]),
+    (1.4, [0, 1, 3, 4, 6, 6, 6, 8, 10]),   # cap = floor(1.4 * 6 * 2 / 8) = 2
+])
+def test_glossary_example_permutation(torch_cuda, capacity_factor, expect_offsets):
+    torch = torch_cuda
+    import sparse_mixture_experts_rmsnorm_b200 as moe
+    fx = json.load(open(os.path.join(GOLDEN, "glossary_top2_example.json")))
+    N, E, k, d = fx["n_tokens"], fx["n_experts"], fx["top_k"], 16
+    lc = moe.Config(N, d, E, k, 16, dtype="bf16", capacity_factor=capacity_factor)
+    ws = moe.workspace(lc)
+    idx = torch.tensor(fx["experts_per_token"], dtype=torch.int32, device="cuda")
+    xn = torch.arange(N * d, dtype=torch.float32, device="cuda").reshape(N, d).to(torch.bfloat16)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device="cuda")
+    slot_row = torch.empty(N * k, dtype=torch.int32, device="cuda")
+    row_token = torch.empty(N * k, dtype=torch.int32, device="cuda")
+    x_perm = torch.zeros(N * k, d, dtype=torch.bfloat16, device="cuda")
+    moe.moe_permute(lc, idx, xn, offsets, slot_row, row_token, x_perm, ws)
+    torch.cuda.synchronize()
+    off = offsets.cpu().tolist()
+    assert off == expect_offsets
+    cap = lc.capacity
+    ref_off, ref_slot, ref_rt = oracle.permute(np.array(fx["experts_per_token"]), E, cap)
+    assert off == ref_off.tolist()
+    assert slot_row.cpu().tolist() == ref_slot.tolist()
+    assert row_token.cpu().tolist()[: off[-1]] == ref_rt.tolist()
+    rows = x_perm[: off[-1]].float().cpu().numpy()
+    np.testing.assert_array_equal(rows, xn.float().cpu().numpy()[ref_rt])
+
+
+# ----------------------------------------------------------------- tcgen05 grouped GEMM, ragged shapes
+
+def _ffn_case(torch, groups_rows, d, H, seed, with_offsets=True):
+    import sparse_mixture_experts_rmsnorm_b200 as moe
+    G = len(groups_rows)
+    R = int(sum(groups_rows))
+    r = np.random.default_rng(seed)
+    bf = lambda a: oracle.round_to(a, "bf16")
+    x = bf(r.standard_normal((R + 7, d)))
+    wg = bf(r.standard_normal((G, H, d)) * 0.05)
+    wu = bf(r.standard_normal((G, H, d)) * 0.05)
+    wd = bf(r.standard_normal((G, d, H)) * 0.05)
+    dev = lambda a: torch.tensor(a, dtype=torch.float32, device="cuda").to(torch.bfloat16).contiguous()
+    lc = moe.Config(n_tokens=max(R, 1), d_model=d, n_experts=G, top_k=1, d_ff=H, dtype="bf16")
+    ws = moe.workspace(lc)
+    offs = np.concatenate([[0], np.cumsum(groups_rows)]).astype(np.int32)
+    y = torch.full((R + 7, d), 77.0, dtype=torch.bfloat16, device="cuda")
+    moe.moe_expert_ffn(lc, G, torch.tensor(offs, device="cuda") if with_offsets else None, R, dev(x), dev(wg),
+                       dev(wu), dev(wd), H, y, ws)
+    torch.cuda.synchronize()
+    st, info = moe.moe_check_device_error(ws)
+    assert st == 0, info
+    got = to_np(y)
+    ref = np.zeros((R, d))
+    for g in range(G):
+        a, b = offs[g], offs[g + 1]
+        if b > a:
+            ref[a:b] = oracle.swiglu_expert(x[a:b], wg[g], wu[g], wd[g], "bf16")
+    assert np.all(got[R:] == 77.0), "rows past the last group were written"
+    return got[:R], ref
+
+
+@pytest.mark.parametrize("rows,d,H", [
+    ([0, 130, 77, 1, 256], 192, 200),      # ragged groups, empty group, partial tiles, 3 k-blocks
+    ([300], 4096, 512),                    # one group, many k-blocks
+    ([5, 0, 0, 129, 64], 520, 1032),       # K and N not multiples of the tile
+])
+def test_expert_ffn_tc_matches_oracle(torch_cuda, rows, d, H):
+    got, ref = _ffn_case(torch_cuda, rows, d, H, seed=len(rows) + d)
+    err = rel_rms_err(got, ref)
+    assert err <= BF16_REL_RMS, err
+    assert err <= 1.5e-2, err
+
+
+def test_expert_ffn_tc_single_group_smaller_than_a_tile(torch_cuda):
+    got, ref = _ffn_case(torch_cuda, [64], 256, 256, seed=5, with_offsets=False)
+    assert rel_rms_err(got, ref) <= BF16_REL_RMS
+
+
+# ----------------------------------------------------------------- router on the tensor cores
+
+@pytest.mark.parametrize("E,k", [(64, 6), (256, 8)])
+def test_router_tc_routing_bit_exact(torch_cuda, E, k):
+    cfg = mi.LayerConfig(name="router", n_tokens=777, d_model=1024, n_experts=E, top_k=k, d_ff=64,
+                         bias=("uniform", -0.01, 0.01), seed=3)
+    g = run_gpu_layer(cfg)
+    ref = oracle_routing(cfg)
+    np.testing.assert_array_equal(g["xn"], ref["xn"])
+    np.testing.assert_allclose(g["scores"], ref["scores"], rtol=2e-5, atol=1e-9)
+    skipped = check_routing(g, ref, k)
+    assert skipped < 0.02 * cfg.n_tokens
+    check_permutation(g, E, -1)
+
+
+# ----------------------------------------------------------------- bias update
+
+def test_bias_update_bit_exact(torch_cuda):
+    torch = torch_cuda
+    import sparse_mixture_experts_rmsnorm_b200 as moe
+    r = np.random.default_rng(7)
+    E = 300
+    counts = r.integers(0, 2048, size=E).astype(np.int32)
+    counts[:5] = 1024
+    bias = (r.standard_normal(E) * 1e-2).astype(np.float32)
+    b = torch.tensor(bias, device="cuda")
+    moe.moe_bias_update(E, torch.tensor(counts, device="cuda"), 1024.0, 1e-3, b)
+    got = b.cpu().numpy()
+    ref = oracle.bias_update(bias, counts, 1024.0, 1e-3)
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+# ----------------------------------------------------------------- bounded device wait
+
+def test_device_wait_times_out_and_reports(torch_cuda):
+    torch = torch_cuda
+    import sparse_mixture_experts_rmsnorm_b200 as moe
+    ws = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    moe.moe_set_wait_timeout_ns(2_000_000)  # 2 ms
+    try:
+        moe.moe_selftest_wait_timeout(ws)
+        st, info = moe.moe_check_device_error(ws)
+    finally:
+        moe.moe_set_wait_timeout_ns(2_000_000_000)
+    assert st == moe.MOE_ERR_DEVICE_TIMEOUT
+    assert info[0] == moe.MOE_ERR_DEVICE_TIMEOUT and info[1] == 2
+    st, info = moe.moe_check_device_error(ws)
+    assert st == 0 and info[0] == 0
+    # the context is still usable
+    x = torch.ones(16, device="cuda")
+    assert float(x.sum()) == 16.0
