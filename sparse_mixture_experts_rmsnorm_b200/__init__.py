@@ -124,6 +124,15 @@ def _stream(stream):
     return stream.cuda_stream
 
 
+def _torch_stream(stream):
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream()
+    if isinstance(stream, int):
+        return torch.cuda.ExternalStream(stream)
+    return stream
+
+
 def _check(status: int, where: str):
     if status != MOE_OK:
         raise MoEError(status, where)
@@ -219,8 +228,13 @@ def moe_layer_forward(cfg: Config, weights: dict, h, bias, out, ws, routing: dic
                          ("scores", "topk_idx", "topk_gate", "counts", "offsets", "slot_row", "row_token")])
     tr = None
     if trace is not None:
-        tr = MoeTrace(*[(trace[n].cuda_event if trace.get(n) is not None else None) for n in
-                        ("start", "routed", "permuted", "gate_up", "down", "shared", "combined")])
+        handles = []
+        for n in ("start", "routed", "permuted", "gate_up", "down", "shared", "combined"):
+            ev = trace.get(n)
+            if ev is not None and not ev.cuda_event:
+                ev.record(_torch_stream(stream))  # torch creates its events lazily, on the first record
+            handles.append(ev.cuda_event if ev is not None else None)
+        tr = MoeTrace(*handles)
     _check(_lib.moe_layer_forward(ctypes.byref(cfg.c()), ctypes.byref(w), _ptr(h), _ptr(bias), _ptr(out),
                                   ctypes.byref(r) if r is not None else None,
                                   ctypes.byref(tr) if tr is not None else None,

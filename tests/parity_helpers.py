@@ -163,4 +163,21 @@ def oracle_outputs(cfg: mi.LayerConfig, ref: dict, tokens, idx, gates, keep) -> 
 
 
 def rel_rms_err(got: np.ndarray, ref: np.ndarray) -> float:
+    """max |got - ref| / rms(ref)."""
     return float(np.max(np.abs(got - ref)) / np.sqrt(np.mean(ref ** 2)))
+
+
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    """Half the bf16 spacing at |x|: the largest error of rounding an exact
+    value to bf16 storage (8 significant bits: x in [2^e, 2^(e+1)) has
+    spacing 2^(e-7))."""
+    _, e = np.frexp(np.abs(np.asarray(x, dtype=np.float64)))  # |x| = m 2^e, 0.5 <= m < 1
+    return np.ldexp(1.0, e - 9)
+
+
+def bf16_rel_rms_err(got: np.ndarray, ref64: np.ndarray) -> float:
+    """Error of a bf16-stored result against the unrounded float64 oracle,
+    beyond the half-ulp that storing even the exact value in bf16 costs:
+    max(0, |got - ref| - half_ulp(ref)) / rms(ref)."""
+    excess = np.maximum(np.abs(got - ref64) - bf16_half_ulp(ref64), 0.0)
+    return float(np.max(excess) / np.sqrt(np.mean(ref64 ** 2)))

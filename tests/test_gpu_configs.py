@@ -9,8 +9,8 @@ import pytest
 
 import moe_inputs as mi
 import oracle
-from parity_helpers import (BF16_REL_RMS, check_permutation, check_routing, oracle_outputs, oracle_routing,
-                            rel_rms_err, run_gpu_layer, tie_masks, to_np)
+from parity_helpers import (BF16_REL_RMS, bf16_rel_rms_err, check_permutation, check_routing, oracle_outputs,
+                            oracle_routing, rel_rms_err, run_gpu_layer, tie_masks, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -51,10 +51,14 @@ def test_config_parity(name):
                                                               replace=False)]))
     ref_out = oracle_outputs(cfg, ref, tokens, ref["idx"], ref["gates"], ref_keep)
     got = g["out"][tokens]
-    err = rel_rms_err(got, ref_out)
-    err_delta = rel_rms_err(got - ref["h"][tokens], ref_out - ref["h"][tokens])
-    print(f"{name}: max|err|/rms(out) = {err:.3e}, on out-h = {err_delta:.3e}, tokens {tokens.size}, "
-          f"skipped ties {skipped}, dropped slots {int((~gpu_keep).sum())}")
+    # the tolerance bounds the arithmetic; storing out in bf16 adds up to half
+    # a bf16 spacing on top of it even for an exact result
+    err = bf16_rel_rms_err(got, ref_out)
+    raw = rel_rms_err(got, ref_out)
+    raw_delta = rel_rms_err(got - ref["h"][tokens], ref_out - ref["h"][tokens])
+    print(f"{name}: beyond-storage max err/rms(out) = {err:.3e}; raw max|err|/rms(out) = {raw:.3e}, "
+          f"on out-h = {raw_delta:.3e}; tokens {tokens.size}, skipped ties {skipped}, "
+          f"dropped slots {int((~gpu_keep).sum())}")
     assert err <= BF16_REL_RMS, err
 
     if cap >= 0:

