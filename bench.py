@@ -36,7 +36,8 @@ UNIT = "tokens/s"
 # DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu
 # capture, with the sha256 of the kernel source it was taken on; reported
 # only while the source is unchanged.
-TRAFFIC = {}
+TRAFFIC = {"kernel_sha": "6c237c8653416339", "workload": "mixtral_bf16", "bytes": 2225753440,
+           "source": "profiles/gemm_tc_swiglu_mixtral_bf16.md"}
 
 
 def _peaks():
