@@ -1,6 +1,7 @@
 """Build libmoe_b200.so (the CUDA kernels and the C ABI) in place, for sm_100a.
 
-Usage:  python -m sparse_mixture_experts_rmsnorm_b200.build [-v]
+Usage:  python sparse_mixture_experts_rmsnorm_b200/build.py [-v] [--ptxas]
+(run as a script: importing the package would load the library first)
 Each .cu under csrc/ is compiled with nvcc in parallel and the objects are
 linked into one shared library next to this file.  Objects are rebuilt only
 when a source or header is newer than the library.
