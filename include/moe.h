@@ -154,6 +154,32 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const voi
                        int32_t* slot_row, int32_t* row_token, void* x_perm, void* ws, size_t ws_bytes,
                        void* stream);
 
+/* Maximum histogram entries, E * ceil(N*k / 256), that moe_permute_noalloc
+ * can handle: 262144 int32 (1 MiB). */
+#define MOE_NOALLOC_HIST_INTS 262144
+
+/* moe_permute without a workspace, for callers that cannot hand the library
+ * device memory for scratch: a plugin or callback that only receives its
+ * own input and output buffers, or a loop that must not allocate once it is
+ * running (cudaMalloc can synchronise the device and take unbounded time).
+ * The pages have no counterpart to this call; it is a deployment variant of
+ * moe_permute.
+ *
+ * Arguments, results and errors are those of moe_permute, minus ws/ws_bytes.
+ * The chunk histograms live in a fixed 1 MiB device array inside the
+ * library instead; every GPU that loads the library holds it until the
+ * process exits.  Rules:
+ *  - E * ceil(N*k / 256) must not exceed MOE_NOALLOC_HIST_INTS, else the
+ *    call returns MOE_ERR_WORKSPACE and enqueues nothing;
+ *  - the first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) and caches it; make that first call before any
+ *    stream capture;
+ *  - every call on a device shares the one array: calls that overlap on the
+ *    GPU (other streams, other threads) race and give wrong results.
+ * The call allocates nothing and frees nothing. */
+moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* topk_idx, const void* xn, int32_t* offsets,
+                               int32_t* slot_row, int32_t* row_token, void* x_perm, void* stream);
+
 /* Steps a6-a8: grouped SwiGLU expert FFN, y = W_down(silu(W_gate x) * (W_up x)).
  * Lesson "The concept" (each expert an independent FFN, usually SwiGLU);
  * "Expert parallelism for MoE serving", "Future" (GEMM units that batch many

@@ -31,7 +31,7 @@ MOE_F32, MOE_BF16 = 0, 1
 # Every entry point declared in include/moe.h, in declaration order.
 ENTRY_POINTS = (
     "moe_status_string", "moe_version", "moe_workspace_size", "moe_workspace_init", "moe_route",
-    "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_bias_update",
+    "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_bias_update",
     "moe_check_device_error", "moe_set_wait_timeout_ns", "moe_selftest_wait_timeout",
 )
 
@@ -66,7 +66,7 @@ class MoeTrace(ctypes.Structure):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m sparse_mixture_experts_rmsnorm_b200.build`")
+                          "`python sparse_mixture_experts_rmsnorm_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     P, I32, I64, SZ, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
     cfgp = ctypes.POINTER(MoeConfig)
@@ -77,6 +77,7 @@ def _load():
         "moe_workspace_init": (I32, [P, SZ, P]),
         "moe_route": (I32, [cfgp, P, P, P, P, P, P, P, P, P, P, SZ, P]),
         "moe_permute": (I32, [cfgp, P, P, P, P, P, P, P, SZ, P]),
+        "moe_permute_noalloc": (I32, [cfgp, P, P, P, P, P, P, P]),
         "moe_expert_ffn": (I32, [cfgp, I32, P, I32, P, P, P, P, I32, P, P, SZ, P]),
         "moe_combine": (I32, [cfgp, P, P, P, P, P, P, P]),
         "moe_layer_forward": (I32, [cfgp, ctypes.POINTER(MoeWeights), P, P, P, ctypes.POINTER(MoeRouting),
@@ -197,6 +198,13 @@ def moe_route(cfg: Config, h, norm_w, w_router, bias, xn, scores, topk_idx, topk
 def moe_permute(cfg: Config, topk_idx, xn, offsets, slot_row, row_token, x_perm, ws, stream=None):
     _check(_lib.moe_permute(ctypes.byref(cfg.c()), _ptr(topk_idx), _ptr(xn), _ptr(offsets), _ptr(slot_row),
                             _ptr(row_token), _ptr(x_perm), _ptr(ws), ws.numel(), _stream(stream)), "moe_permute")
+
+
+def moe_permute_noalloc(cfg: Config, topk_idx, xn, offsets, slot_row, row_token, x_perm, stream=None):
+    """moe_permute without a workspace (the histograms use the library's fixed
+    1 MiB device array; calls that overlap on the GPU race)."""
+    _check(_lib.moe_permute_noalloc(ctypes.byref(cfg.c()), _ptr(topk_idx), _ptr(xn), _ptr(offsets), _ptr(slot_row),
+                                    _ptr(row_token), _ptr(x_perm), _stream(stream)), "moe_permute_noalloc")
 
 
 def moe_expert_ffn(cfg: Config, n_groups: int, offsets, max_rows: int, x, w_gate, w_up, w_down, d_ff: int, y, ws,

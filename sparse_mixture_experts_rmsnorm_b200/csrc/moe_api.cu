@@ -38,7 +38,7 @@ struct Layout {
   int64_t act_elems; // max(R * H, N * Hs)
 };
 
-static int64_t capacity_of(const moe_config* c) {
+int64_t capacity_of(const moe_config* c) {
   if (!(c->capacity_factor > 0.f)) return -1;
   return (int64_t)floor((double)c->capacity_factor * (double)c->n_tokens * (double)c->top_k / (double)c->n_experts);
 }
@@ -77,7 +77,7 @@ static Layout layout_of(const moe_config* c) {
   return L;
 }
 
-static bool config_ok(const moe_config* c) {
+bool config_ok(const moe_config* c) {
   if (c == nullptr) return false;
   if (c->n_tokens < 0 || c->d_model < 1 || c->n_experts < 1 || c->n_experts > 1024) return false;
   if (c->top_k < 1 || c->top_k > c->n_experts || c->top_k > 32) return false;
@@ -90,7 +90,7 @@ static bool config_ok(const moe_config* c) {
 
 // Shapes the kernels do not cover: bf16 rows must be whole 16-byte units for
 // TMA (d % 8 == 0, H % 8 == 0, Hs % 8 == 0).
-static bool config_supported(const moe_config* c) {
+bool config_supported(const moe_config* c) {
   if (c->dtype == MOE_BF16) {
     if (c->d_model % 8 || c->d_ff % 8 || c->d_ff_shared % 8) return false;
   }

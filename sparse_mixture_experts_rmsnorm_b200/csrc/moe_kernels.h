@@ -10,6 +10,11 @@
 
 namespace moe_host {
 
+// Config checks and the capacity rule shared by the entry points (moe_api.cu).
+bool config_ok(const moe_config* c);          // sizes and dtype valid
+bool config_supported(const moe_config* c);   // covered by the kernels
+int64_t capacity_of(const moe_config* c);     // floor(C*N*k/E), or -1 without a capacity
+
 // a1: xn = RMSNorm(h) (one block per token).
 moe_status launch_rmsnorm(int dtype, const void* h, const void* norm_w, void* xn, int n, int d, float eps,
                           cudaStream_t s);
