@@ -123,6 +123,19 @@ def workload_flops_bytes(cfg, offsets_host=None):
             "expert_flops": gate_up + down + shared}
 
 
+def workload(args):
+    """The named workload, with any --set key=value overrides applied (used to
+    profile a smaller case of the same per-expert shape)."""
+    import moe_inputs as mi
+    cfg = mi.CONFIGS[args.workload]
+    over = {}
+    for kv in args.set or []:
+        k, v = kv.split("=", 1)
+        cur = getattr(cfg, k)
+        over[k] = type(cur)(v) if not isinstance(cur, bool) else v.lower() in ("1", "true")
+    return cfg.with_(**over) if over else cfg
+
+
 def run_native(args):
     import torch
     import torch.distributed as dist
@@ -134,7 +147,7 @@ def run_native(args):
     torch.cuda.set_device(local)
     if world > 1:
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
-    cfg = mi.CONFIGS[args.workload]
+    cfg = workload(args)
     lc = moe.Config(cfg.n_tokens, cfg.d_model, cfg.n_experts, cfg.top_k, cfg.d_ff, cfg.d_ff_shared, cfg.dtype,
                     cfg.rms_eps, cfg.capacity_factor)
     # each replica gets its own tokens (seed = rank), the same weights (seed 0)
@@ -246,7 +259,8 @@ def run_native(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "f32",
             "data": "synthetic (seeded counter-hash generator; random-init weights of the layer's shapes)",
-            "config": {"workload": args.workload, "n_tokens": cfg.n_tokens, "d_model": cfg.d_model,
+            "config": {"workload": args.workload + ("" if not args.set else " with " + ",".join(args.set)),
+                       "n_tokens": cfg.n_tokens, "d_model": cfg.d_model,
                        "n_experts": cfg.n_experts, "top_k": cfg.top_k, "d_ff": cfg.d_ff,
                        "d_ff_shared": cfg.d_ff_shared, "capacity_factor": cfg.capacity_factor,
                        "parallelism": f"replicas x{world} (token-sharded, no exchange)",
@@ -326,8 +340,7 @@ def run_reference(args):
     world, rank, _ = _dist()
     if rank != 0:
         return
-    import moe_inputs as mi
-    cfg = mi.CONFIGS[args.workload]
+    cfg = workload(args)
     # each step a bounded sample: the whole run stays near two minutes
     n_tok = _calibrated_tokens(cfg, 120.0 / (args.steps + args.warmup))
     sub, a = _oracle_sample(cfg, n_tok)
@@ -359,6 +372,8 @@ def main():
     ap.add_argument("--workload", default="mixtral_bf16")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--set", action="append", metavar="KEY=VALUE",
+                    help="override a workload field, e.g. --set n_experts=32 --set n_tokens=1024")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

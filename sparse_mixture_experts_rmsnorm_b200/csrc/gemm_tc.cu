@@ -132,6 +132,27 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 
 __device__ __forceinline__ float silu_tc(float z) { return __fdiv_rn(z, __fadd_rn(1.f, expf(-z))); }
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);  // .x = lo (lower address), .y = hi
+  return *reinterpret_cast<uint32_t*>(&p);
+}
+
+// Store 32 consecutive columns [col, col + 32) of one output row as bf16,
+// masked to col < nout; 16-byte stores when the row allows them.
+__device__ __forceinline__ void store_row32_bf16(bf16* out, int col, int nout, bool vec_ok, const float (&v)[32]) {
+  if (vec_ok && col + 32 <= nout) {
+    uint4* dst = reinterpret_cast<uint4*>(out + col);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      dst[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                          pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (col + i < nout) out[col + i] = __float2bfloat16_rn(v[i]);
+  }
+}
+
 // ---- tile schedule -----------------------------------------------------------
 struct Tile {
   int group, row0, row_end, n0;
@@ -342,20 +363,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           MOE_TMEM_LD32(tbase + c, g);
           MOE_TMEM_LD32(tbase + 128 + c, u);
           tmem_wait_ld();
-          __align__(16) bf16 o[32];
+          float v[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            o[i] = __float2bfloat16_rn(__fmul_rn(silu_tc(__uint_as_float(g[i])), __uint_as_float(u[i])));
-          const int col = tl.n0 + c;
-          if (row_ok) {
-            if (col + 32 <= args.nout && (args.ldc & 7) == 0) {
-              uint4* dst = reinterpret_cast<uint4*>(out + col);
-#pragma unroll
-              for (int v = 0; v < 4; ++v) dst[v] = reinterpret_cast<const uint4*>(o)[v];
-            } else {
-              for (int i = 0; i < 32 && col + i < args.nout; ++i) out[col + i] = o[i];
-            }
-          }
+          for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(silu_tc(__uint_as_float(g[i])), __uint_as_float(u[i]));
+          if (row_ok) store_row32_bf16(out, tl.n0 + c, args.nout, (args.ldc & 7) == 0, v);
         }
       } else {
 #pragma unroll 1
@@ -370,22 +381,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               if (col + 32 <= args.nout && (args.ldc & 3) == 0) {
                 uint4* dst = reinterpret_cast<uint4*>(out + col);
 #pragma unroll
-                for (int v = 0; v < 8; ++v) dst[v] = make_uint4(a[4 * v], a[4 * v + 1], a[4 * v + 2], a[4 * v + 3]);
+                for (int q = 0; q < 8; ++q) dst[q] = make_uint4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
               } else {
-                for (int i = 0; i < 32 && col + i < args.nout; ++i) out[col + i] = __uint_as_float(a[i]);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                  if (col + i < args.nout) out[col + i] = __uint_as_float(a[i]);
               }
             } else {
-              bf16* out = reinterpret_cast<bf16*>(args.C) + (size_t)row * args.ldc;
-              __align__(16) bf16 o[32];
+              float v[32];
 #pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = __float2bfloat16_rn(__uint_as_float(a[i]));
-              if (col + 32 <= args.nout && (args.ldc & 7) == 0) {
-                uint4* dst = reinterpret_cast<uint4*>(out + col);
-#pragma unroll
-                for (int v = 0; v < 4; ++v) dst[v] = reinterpret_cast<const uint4*>(o)[v];
-              } else {
-                for (int i = 0; i < 32 && col + i < args.nout; ++i) out[col + i] = o[i];
-              }
+              for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(a[i]);
+              store_row32_bf16(reinterpret_cast<bf16*>(args.C) + (size_t)row * args.ldc, col, args.nout,
+                               (args.ldc & 7) == 0, v);
             }
           }
         }

@@ -89,11 +89,12 @@ bool config_ok(const moe_config* c) {
 }
 
 // Shapes the kernels do not cover: bf16 rows must be whole 16-byte units for
-// TMA (d % 8 == 0, H % 8 == 0, Hs % 8 == 0).
+// TMA (d % 8 == 0, H % 8 == 0, Hs % 8 == 0), and d <= 49152.
 bool config_supported(const moe_config* c) {
   if (c->dtype == MOE_BF16) {
     if (c->d_model % 8 || c->d_ff % 8 || c->d_ff_shared % 8) return false;
   }
+  if (c->d_model > 49152) return false;  // RMSNorm stages one fp32 row in shared memory
   return true;
 }
 
@@ -115,14 +116,10 @@ static moe_status check_common(const moe_config* c, const void* ws, size_t ws_by
 
 static inline char* wsp(void* ws, size_t off) { return static_cast<char*>(ws) + off; }
 
-// a2: router logits [N][E] fp32 = xn . W_router^T
-static moe_status router_logits(const moe_config* c, const void* xn, const void* w_router, float* logits,
-                                int32_t* hdr, cudaStream_t s) {
-  if (use_tc(c) && c->n_experts >= 64)
-    return launch_gemm_tc(EPI_F32, xn, w_router, nullptr, nullptr, 1, c->n_tokens, c->n_experts, c->d_model, logits,
-                          c->n_experts, hdr, s);
-  return launch_gemm_simt(c->dtype, EPI_F32, xn, w_router, nullptr, nullptr, 1, c->n_tokens, c->n_experts,
-                          c->d_model, logits, c->n_experts, s);
+// a2 on the tensor cores pays off once there are many tokens and experts;
+// below that the router dot products ride along with RMSNorm.
+static bool router_on_tc(const moe_config* c) {
+  return use_tc(c) && c->n_experts >= 64 && c->n_tokens >= 512;
 }
 
 static moe_status route_impl(const moe_config* c, const void* h, const void* norm_w, const void* w_router,
@@ -131,8 +128,17 @@ static moe_status route_impl(const moe_config* c, const void* h, const void* nor
   const Layout L = layout_of(c);
   int32_t* hdr = (int32_t*)wsp(ws, L.hdr);
   float* logits = (float*)wsp(ws, L.logits);
-  MOE_TRY(launch_rmsnorm(c->dtype, h, norm_w, xn, c->n_tokens, c->d_model, c->rms_eps, s));
-  if (c->n_tokens > 0) MOE_TRY(router_logits(c, xn, w_router, logits, hdr, s));
+  if (c->n_tokens > 0) {
+    if (router_on_tc(c)) {
+      MOE_TRY(launch_rmsnorm_router(c->dtype, h, norm_w, nullptr, xn, nullptr, c->n_tokens, c->d_model,
+                                    c->n_experts, c->rms_eps, s));
+      MOE_TRY(launch_gemm_tc(EPI_F32, xn, w_router, nullptr, nullptr, 1, c->n_tokens, c->n_experts, c->d_model,
+                             logits, c->n_experts, hdr, s));
+    } else {
+      MOE_TRY(launch_rmsnorm_router(c->dtype, h, norm_w, w_router, xn, logits, c->n_tokens, c->d_model,
+                                    c->n_experts, c->rms_eps, s));
+    }
+  }
   return launch_topk(logits, bias, scores, topk_idx, topk_gate, counts, c->n_tokens, c->n_experts, c->top_k, s);
 }
 

@@ -15,9 +15,11 @@ bool config_ok(const moe_config* c);          // sizes and dtype valid
 bool config_supported(const moe_config* c);   // covered by the kernels
 int64_t capacity_of(const moe_config* c);     // floor(C*N*k/E), or -1 without a capacity
 
-// a1: xn = RMSNorm(h) (one block per token).
-moe_status launch_rmsnorm(int dtype, const void* h, const void* norm_w, void* xn, int n, int d, float eps,
-                          cudaStream_t s);
+// a1: xn = RMSNorm(h), and with logits != nullptr also a2 on the CUDA
+// cores: logits [N][E] fp32 = xn . W_router^T (one block per token and
+// group of up to 32 experts).  d * 4 bytes of shared memory per block.
+moe_status launch_rmsnorm_router(int dtype, const void* h, const void* norm_w, const void* w_router, void* xn,
+                                 float* logits, int n, int d, int e, float eps, cudaStream_t s);
 
 // a3: softmax over the router logits, top-k on score + bias, renormalised
 // gates and the per-expert counts (counts are zeroed here first).

@@ -1,5 +1,6 @@
-// Steps a1 and a3 of the MoE layer: RMSNorm, and the router's softmax,
-// top-k on score + bias with gates from the raw scores, and expert counts.
+// Steps a1-a3 of the MoE layer: RMSNorm (with the router dot products on
+// the CUDA cores when that is the faster place for them), and the router's
+// softmax, top-k on score + bias with gates from the raw scores, and counts.
 //
 // Sources: "Mixture of Experts (MoE)" lesson (AI Engineering from Scratch,
 // Phase 07), "The concept / Swapping the FFN" (one norm(h) feeds the router
@@ -8,30 +9,63 @@
 // wins a tie) and "The load-balancing problem" (DeepSeek-V3: bias changes
 // selection only); Ultralytics glossary "Mixture of Experts (MoE)", "How an
 // MoE layer works" (outputs weighted by the normalised router scores).
-// The router logits themselves come from the grouped GEMM kernels.
+// With many experts and many tokens the router logits come from the tcgen05
+// grouped GEMM instead.
 #include "moe_common.cuh"
 #include "moe_kernels.h"
 
 namespace moe {
 
 // ---------------------------------------------------------------------------
-// a1. RMSNorm: xn = h / sqrt(mean(h^2) + eps) * w.
+// a1 (+ a2 on the CUDA cores). RMSNorm: xn = h / sqrt(mean(h^2) + eps) * w.
 // mean(h^2) is summed in fp64 (every h^2 is exact there); the scale
 // r = fl32(1 / sqrt(ms + eps)) is taken in fp64 and rounded once, then
 // xn = round(fl32(fl32(h * r) * w)), so the storage rounding is decided in fp32.
-// One block per token, grid-stride over tokens.
+//
+// One block per token (grid-stride), V elements per 16-byte access.  The
+// row is staged in shared memory as fp32; when `logits` is given, the
+// block's warps then take the router dot products of the rounded xn row
+// with experts [e0, e0 + epb) (e0 = blockIdx.y * epb), one expert per warp
+// at a time, fp32 FMA per lane and a warp tree sum.  Blocks with
+// blockIdx.y == 0 write xn.
 // ---------------------------------------------------------------------------
-template <typename T>
-__global__ void __launch_bounds__(256) rmsnorm_kernel(const T* __restrict__ h, const T* __restrict__ w,
-                                                      T* __restrict__ xn, int n, int d, float eps) {
+template <typename T, int V>
+struct Vec {
+  static_assert(V * sizeof(T) == 16 || V == 1, "V elements must fill 16 bytes");
+  T v[V];
+};
+
+template <typename T, int V>
+__device__ __forceinline__ void load_vec(const T* p, float (&f)[V]) {
+  Vec<T, V> x;
+  if (V * sizeof(T) == 16) *reinterpret_cast<uint4*>(&x) = *reinterpret_cast<const uint4*>(p);
+  else x.v[0] = p[0];
+#pragma unroll
+  for (int j = 0; j < V; ++j) f[j] = to_f32(x.v[j]);
+}
+
+template <typename T, int V>
+__global__ void __launch_bounds__(256) rmsnorm_router_kernel(const T* __restrict__ h, const T* __restrict__ w,
+                                                             const T* __restrict__ w_router, T* __restrict__ xn,
+                                                             float* __restrict__ logits, int n, int d, int E,
+                                                             int epb, float eps) {
+  extern __shared__ float row[];  // d floats
   __shared__ double part[8];
   __shared__ float r_sh;
+  const int e0 = blockIdx.y * epb;
+  const int e1 = min(E, e0 + epb);
+  const int warps = blockDim.x >> 5;
   for (int t = blockIdx.x; t < n; t += gridDim.x) {
-    const T* row = h + (size_t)t * d;
+    const T* hr = h + (size_t)t * d;
     double acc = 0.0;
-    for (int i = threadIdx.x; i < d; i += blockDim.x) {
-      double v = (double)to_f32(row[i]);
-      acc += v * v;
+    for (int i = threadIdx.x * V; i < d; i += blockDim.x * V) {
+      float f[V];
+      load_vec<T, V>(hr + i, f);
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        acc += (double)f[j] * (double)f[j];
+        row[i + j] = f[j];
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -39,16 +73,41 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const T* __restrict__ h, c
     __syncthreads();
     if (threadIdx.x == 0) {
       double s = 0.0;
-      for (int i = 0; i < (int)(blockDim.x >> 5); ++i) s += part[i];
-      double ms = s / (double)d;
-      r_sh = (float)(1.0 / sqrt(ms + (double)eps));
+      for (int i = 0; i < warps; ++i) s += part[i];
+      r_sh = (float)(1.0 / sqrt(s / (double)d + (double)eps));
     }
     __syncthreads();
     const float r = r_sh;
-    T* out = xn + (size_t)t * d;
-    for (int i = threadIdx.x; i < d; i += blockDim.x) {
-      float v = __fmul_rn(__fmul_rn(to_f32(row[i]), r), to_f32(w[i]));
-      out[i] = from_f32<T>(v);
+    const bool store = (blockIdx.y == 0) && xn != nullptr;
+    for (int i = threadIdx.x * V; i < d; i += blockDim.x * V) {
+      float wf[V];
+      load_vec<T, V>(w + i, wf);
+      Vec<T, V> q;
+#pragma unroll
+      for (int j = 0; j < V; ++j) {
+        q.v[j] = from_f32<T>(__fmul_rn(__fmul_rn(row[i + j], r), wf[j]));
+        row[i + j] = to_f32(q.v[j]);
+      }
+      if (store) {
+        if (V * sizeof(T) == 16) *reinterpret_cast<uint4*>(xn + (size_t)t * d + i) = *reinterpret_cast<uint4*>(&q);
+        else xn[(size_t)t * d + i] = q.v[0];
+      }
+    }
+    __syncthreads();
+    if (logits != nullptr) {
+      for (int e = e0 + warp_id(); e < e1; e += warps) {
+        const T* wr = w_router + (size_t)e * d;
+        float s = 0.f;
+        for (int i = lane_id() * V; i < d; i += 32 * V) {
+          float wf[V];
+          load_vec<T, V>(wr + i, wf);
+#pragma unroll
+          for (int j = 0; j < V; ++j) s = __fmaf_rn(row[i + j], wf[j], s);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane_id() == 0) logits[(size_t)t * E + e] = s;
+      }
     }
     __syncthreads();
   }
@@ -152,17 +211,38 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
 
 namespace moe_host {
 
-moe_status launch_rmsnorm(int dtype, const void* h, const void* norm_w, void* xn, int n, int d, float eps,
-                          cudaStream_t s) {
-  if (n == 0) return MOE_OK;
-  int grid = n < sm_count() * 16 ? n : sm_count() * 16;
-  if (dtype == MOE_BF16)
-    moe::rmsnorm_kernel<moe::bf16><<<grid, 256, 0, s>>>((const moe::bf16*)h, (const moe::bf16*)norm_w,
-                                                        (moe::bf16*)xn, n, d, eps);
-  else
-    moe::rmsnorm_kernel<float><<<grid, 256, 0, s>>>((const float*)h, (const float*)norm_w, (float*)xn, n, d,
-                                                    eps);
+template <typename T, int V>
+static moe_status launch_rr(const void* h, const void* norm_w, const void* w_router, void* xn, float* logits, int n,
+                            int d, int e, float eps, cudaStream_t s) {
+  const size_t smem = sizeof(float) * (size_t)d;
+  auto kern = moe::rmsnorm_router_kernel<T, V>;
+  if (smem > 48 * 1024) {
+    static bool done[64] = {};
+    int dev = current_device();
+    if (dev >= 64 || !done[dev]) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (dev < 64) done[dev] = true;
+    }
+  }
+  const int epb = (logits == nullptr) ? 1 : (e <= 32 ? e : 32);
+  const int yb = (logits == nullptr) ? 1 : (e + epb - 1) / epb;
+  int xb = n < sm_count() * 16 ? n : sm_count() * 16;
+  kern<<<dim3(xb, yb), 256, smem, s>>>((const T*)h, (const T*)norm_w, (const T*)w_router, (T*)xn, logits, n, d, e,
+                                       epb, eps);
   return launch_status();
+}
+
+moe_status launch_rmsnorm_router(int dtype, const void* h, const void* norm_w, const void* w_router, void* xn,
+                                 float* logits, int n, int d, int e, float eps, cudaStream_t s) {
+  if (n == 0) return MOE_OK;
+  const uintptr_t addr = (uintptr_t)h | (uintptr_t)norm_w | (uintptr_t)xn | (uintptr_t)(w_router ? w_router : h);
+  if (dtype == MOE_BF16) {
+    if (d % 8 == 0 && addr % 16 == 0) return launch_rr<moe::bf16, 8>(h, norm_w, w_router, xn, logits, n, d, e, eps, s);
+    return launch_rr<moe::bf16, 1>(h, norm_w, w_router, xn, logits, n, d, e, eps, s);
+  }
+  if (d % 4 == 0 && addr % 16 == 0) return launch_rr<float, 4>(h, norm_w, w_router, xn, logits, n, d, e, eps, s);
+  return launch_rr<float, 1>(h, norm_w, w_router, xn, logits, n, d, e, eps, s);
 }
 
 moe_status launch_topk(const float* logits, const float* bias, float* scores, int32_t* topk_idx,

@@ -262,3 +262,29 @@ def test_device_wait_times_out_and_reports(torch_cuda):
     # the context is still usable
     x = torch.ones(16, device="cuda")
     assert float(x.sum()) == 16.0
+
+
+# ----------------------------------------------------------------- small bf16 layers, every output
+
+@pytest.mark.parametrize("over", [
+    dict(n_tokens=300, d_model=256, n_experts=16, top_k=4, d_ff=192, d_ff_shared=128),
+    dict(n_tokens=515, d_model=512, n_experts=8, top_k=2, d_ff=264, capacity_factor=0.9,
+         skew=(5, 8.0, 2.0)),
+    dict(n_tokens=97, d_model=128, n_experts=64, top_k=6, d_ff=64, d_ff_shared=64,
+         bias=("uniform", -0.01, 0.01)),
+])
+def test_small_bf16_layer_every_output(torch_cuda, over):
+    cfg = mi.LayerConfig(name="small", dtype="bf16", seed=4, **over)
+    g = run_gpu_layer(cfg)
+    ref = _full_oracle(cfg)
+    np.testing.assert_array_equal(g["xn"], ref["xn"])
+    check_routing(g, {"key": ref["key"], "idx": ref["idx"], "gates": ref["gates"], "scores": ref["scores"]},
+                  cfg.top_k)
+    check_permutation(g, cfg.n_experts, cfg.capacity)
+    err = bf16_rel_rms_err(g["out"], ref["out64"])
+    print(f"small bf16 layer {over}: beyond-storage max err/rms {err:.3e}")
+    assert err <= BF16_REL_RMS, err
+    dropped_all = np.nonzero((g["slot_row"].reshape(cfg.n_tokens, cfg.top_k) < 0).all(axis=1))[0]
+    if cfg.d_ff_shared == 0 and dropped_all.size:
+        np.testing.assert_array_equal(g["out"][dropped_all], ref["h"][dropped_all] if "h" in ref else
+                                      mi.host_tensor(cfg, "h")[dropped_all])
