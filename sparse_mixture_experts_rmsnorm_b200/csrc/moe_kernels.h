@@ -17,7 +17,7 @@ int64_t capacity_of(const moe_config* c);     // floor(C*N*k/E), or -1 without a
 
 // a1: xn = RMSNorm(h), and with logits != nullptr also a2 on the CUDA
 // cores: logits [N][E] fp32 = xn . W_router^T (one block per token and
-// group of up to 32 experts).  d * 4 bytes of shared memory per block.
+// group of up to 32 experts).  One row of shared memory per block.
 moe_status launch_rmsnorm_router(int dtype, const void* h, const void* norm_w, const void* w_router, void* xn,
                                  float* logits, int n, int d, int e, float eps, cudaStream_t s);
 

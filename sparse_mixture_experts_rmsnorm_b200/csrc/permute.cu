@@ -17,11 +17,11 @@
 // deterministic and equals a stable sort.
 //
 // Kernels: (1) one warp per chunk of 256 slots counts the chunk's slots per
-// expert into hist[e][chunk]; (2) one block scans hist in expert-major order
-// (giving every chunk its starting position within its expert) and forms the
-// kept counts and offsets; (3) the chunk warps recompute their in-chunk ranks
-// and write slot_row / row_token; (4) the gather copies rows with 16-byte
-// loads.
+// expert into hist[e][chunk]; (2) one block scans each expert's row of hist
+// (giving every chunk the rank of its first slot within the expert) and
+// forms the kept counts and offsets; (3) the chunk warps recompute their
+// in-chunk ranks and write slot_row / row_token; (4) the gather copies rows
+// with 16-byte loads.
 #include "moe_common.cuh"
 #include "moe_kernels.h"
 
@@ -66,78 +66,57 @@ __global__ void __launch_bounds__(kPermWarps * 32) chunk_hist_kernel(const int32
   for (int e = lane_id(); e < E; e += 32) hist[(int64_t)e * nchunks + c] = run[e];
 }
 
-// One block of 1024 threads.  Exclusive scan of hist (E*nchunks ints,
-// expert-major) in place, tile by tile with a running carry; then
-//   count_e = start_{e+1} - start_e, kept_e = min(count_e, cap),
-//   offsets = exclusive scan of kept (E+1 entries).
-__global__ void __launch_bounds__(1024) hist_scan_kernel(int32_t* __restrict__ hist, int64_t len, int E,
-                                                         int nchunks, int64_t slots, int cap,
+// One block of 1024 threads.
+//   1. Each warp takes whole experts: the exclusive scan of hist[e][*] over
+//      the chunks, in place, gives every chunk the rank of its first slot of
+//      expert e; the row total is count_e.
+//   2. kept_e = min(count_e, cap); offsets = exclusive scan of kept (E+1).
+__global__ void __launch_bounds__(1024) hist_scan_kernel(int32_t* __restrict__ hist, int E, int nchunks, int cap,
                                                          int32_t* __restrict__ offsets) {
-  constexpr int PER = 8;
-  __shared__ int32_t warp_sum[32];
-  __shared__ int32_t carry_sh;
   __shared__ int32_t kept_sh[1024];
-  const int tid = threadIdx.x;
-  if (tid == 0) carry_sh = 0;
-  __syncthreads();
-  for (int64_t base = 0; base < len; base += 1024 * PER) {
-    int32_t v[PER];
-    int32_t local = 0;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      int64_t p = base + (int64_t)tid * PER + i;
-      v[i] = (p < len) ? hist[p] : 0;
-      local += v[i];
-    }
-    // block-wide exclusive scan of `local`
-    int32_t x = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      int32_t y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane_id() >= o) x += y;
-    }
-    if (lane_id() == 31) warp_sum[warp_id()] = x;
-    __syncthreads();
-    if (warp_id() == 0) {
-      int32_t w = warp_sum[lane_id()];
+  __shared__ int32_t warp_sum[32];
+  const int lane = lane_id(), warp = warp_id();
+  for (int e = warp; e < E; e += 32) {
+    int32_t* row = hist + (int64_t)e * nchunks;
+    int32_t carry = 0;
+    for (int c0 = 0; c0 < nchunks; c0 += 32) {
+      const int c = c0 + lane;
+      const int32_t v = (c < nchunks) ? row[c] : 0;
+      int32_t x = v;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        int32_t y = __shfl_up_sync(0xffffffffu, w, o);
-        if (lane_id() >= o) w += y;
+        int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
       }
-      warp_sum[lane_id()] = w;  // inclusive
+      if (c < nchunks) row[c] = carry + x - v;
+      carry += __shfl_sync(0xffffffffu, x, 31);
     }
-    __syncthreads();
-    int32_t carry = carry_sh;
-    int32_t excl = carry + (x - local) + (warp_id() > 0 ? warp_sum[warp_id() - 1] : 0);
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      int64_t p = base + (int64_t)tid * PER + i;
-      if (p < len) hist[p] = excl;
-      excl += v[i];
-    }
-    __syncthreads();
-    if (tid == 0) carry_sh = carry + warp_sum[31];
-    __syncthreads();
+    if (lane == 0) kept_sh[e] = (cap >= 0 && carry > cap) ? cap : carry;
   }
-  // kept counts and their exclusive scan (E <= 1024: one expert per thread)
-  int32_t kept = 0;
-  if (tid < E) {
-    int32_t start = hist[(int64_t)tid * nchunks];
-    int32_t end = (tid + 1 < E) ? hist[(int64_t)(tid + 1) * nchunks] : (int32_t)slots;
-    kept = end - start;
-    if (cap >= 0 && kept > cap) kept = cap;
-  }
-  kept_sh[tid] = kept;
   __syncthreads();
-  if (tid == 0) {
-    int32_t acc = 0;
-    for (int e = 0; e < E; ++e) {
-      offsets[e] = acc;
-      acc += kept_sh[e];
-    }
-    offsets[E] = acc;
+  const int tid = threadIdx.x;
+  const int32_t k = (tid < E) ? kept_sh[tid] : 0;
+  int32_t x = k;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
   }
+  if (lane == 31) warp_sum[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = warp_sum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sum[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  const int32_t excl = x - k + (warp > 0 ? warp_sum[warp - 1] : 0);
+  if (tid < E) offsets[tid] = excl;
+  if (tid == E - 1) offsets[E] = excl + k;
 }
 
 __global__ void __launch_bounds__(kPermWarps * 32) chunk_scatter_kernel(
@@ -151,7 +130,7 @@ __global__ void __launch_bounds__(kPermWarps * 32) chunk_scatter_kernel(
   __syncwarp();
   if (c >= nchunks) return;
   chunk_walk(idx, slots, c, run, [&](int64_t s, int e, int r_in_chunk) {
-    int32_t rank = hist[(int64_t)e * nchunks + c] - hist[(int64_t)e * nchunks] + r_in_chunk;
+    int32_t rank = hist[(int64_t)e * nchunks + c] + r_in_chunk;
     if (cap < 0 || rank < cap) {
       int32_t row = offsets[e] + rank;
       slot_row[s] = row;
@@ -196,7 +175,7 @@ moe_status launch_permute(const int32_t* topk_idx, int n, int k, int e, int cap,
   const int blocks = (int)((nch + moe::kPermWarps - 1) / moe::kPermWarps);
   const size_t smem = sizeof(int32_t) * e * moe::kPermWarps;
   moe::chunk_hist_kernel<<<blocks, moe::kPermWarps * 32, smem, s>>>(topk_idx, slots, e, (int)nch, hist);
-  moe::hist_scan_kernel<<<1, 1024, 0, s>>>(hist, nch * e, e, (int)nch, slots, cap, offsets);
+  moe::hist_scan_kernel<<<1, 1024, 0, s>>>(hist, e, (int)nch, cap, offsets);
   moe::chunk_scatter_kernel<<<blocks, moe::kPermWarps * 32, smem, s>>>(topk_idx, slots, k, e, (int)nch, cap,
                                                                        hist, offsets, slot_row, row_token);
   return launch_status();

@@ -23,7 +23,7 @@ namespace moe {
 // xn = round(fl32(fl32(h * r) * w)), so the storage rounding is decided in fp32.
 //
 // One block per token (grid-stride), V elements per 16-byte access.  The
-// row is staged in shared memory as fp32; when `logits` is given, the
+// row is staged in shared memory in its own dtype; when `logits` is given, the
 // block's warps then take the router dot products of the rounded xn row
 // with experts [e0, e0 + epb) (e0 = blockIdx.y * epb), one expert per warp
 // at a time, fp32 FMA per lane and a warp tree sum.  Blocks with
@@ -36,12 +36,23 @@ struct Vec {
 };
 
 template <typename T, int V>
-__device__ __forceinline__ void load_vec(const T* p, float (&f)[V]) {
+__device__ __forceinline__ void vec_to_f32(const Vec<T, V>& x, float (&f)[V]) {
+#pragma unroll
+  for (int j = 0; j < V; ++j) f[j] = to_f32(x.v[j]);
+}
+
+template <typename T, int V>
+__device__ __forceinline__ Vec<T, V> ld_vec(const T* p) {
   Vec<T, V> x;
   if (V * sizeof(T) == 16) *reinterpret_cast<uint4*>(&x) = *reinterpret_cast<const uint4*>(p);
   else x.v[0] = p[0];
-#pragma unroll
-  for (int j = 0; j < V; ++j) f[j] = to_f32(x.v[j]);
+  return x;
+}
+
+template <typename T, int V>
+__device__ __forceinline__ void st_vec(T* p, const Vec<T, V>& x) {
+  if (V * sizeof(T) == 16) *reinterpret_cast<uint4*>(p) = *reinterpret_cast<const uint4*>(&x);
+  else p[0] = x.v[0];
 }
 
 template <typename T, int V>
@@ -49,7 +60,8 @@ __global__ void __launch_bounds__(256) rmsnorm_router_kernel(const T* __restrict
                                                              const T* __restrict__ w_router, T* __restrict__ xn,
                                                              float* __restrict__ logits, int n, int d, int E,
                                                              int epb, float eps) {
-  extern __shared__ float row[];  // d floats
+  extern __shared__ __align__(16) uint8_t row_raw[];  // one row of d elements of T
+  T* row = reinterpret_cast<T*>(row_raw);
   __shared__ double part[8];
   __shared__ float r_sh;
   const int e0 = blockIdx.y * epb;
@@ -59,13 +71,12 @@ __global__ void __launch_bounds__(256) rmsnorm_router_kernel(const T* __restrict
     const T* hr = h + (size_t)t * d;
     double acc = 0.0;
     for (int i = threadIdx.x * V; i < d; i += blockDim.x * V) {
+      const Vec<T, V> x = ld_vec<T, V>(hr + i);
       float f[V];
-      load_vec<T, V>(hr + i, f);
+      vec_to_f32(x, f);
 #pragma unroll
-      for (int j = 0; j < V; ++j) {
-        acc += (double)f[j] * (double)f[j];
-        row[i + j] = f[j];
-      }
+      for (int j = 0; j < V; ++j) acc += (double)f[j] * (double)f[j];
+      st_vec<T, V>(row + i, x);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -80,18 +91,14 @@ __global__ void __launch_bounds__(256) rmsnorm_router_kernel(const T* __restrict
     const float r = r_sh;
     const bool store = (blockIdx.y == 0) && xn != nullptr;
     for (int i = threadIdx.x * V; i < d; i += blockDim.x * V) {
-      float wf[V];
-      load_vec<T, V>(w + i, wf);
+      float f[V], wf[V];
+      vec_to_f32(ld_vec<T, V>(row + i), f);
+      vec_to_f32(ld_vec<T, V>(w + i), wf);
       Vec<T, V> q;
 #pragma unroll
-      for (int j = 0; j < V; ++j) {
-        q.v[j] = from_f32<T>(__fmul_rn(__fmul_rn(row[i + j], r), wf[j]));
-        row[i + j] = to_f32(q.v[j]);
-      }
-      if (store) {
-        if (V * sizeof(T) == 16) *reinterpret_cast<uint4*>(xn + (size_t)t * d + i) = *reinterpret_cast<uint4*>(&q);
-        else xn[(size_t)t * d + i] = q.v[0];
-      }
+      for (int j = 0; j < V; ++j) q.v[j] = from_f32<T>(__fmul_rn(__fmul_rn(f[j], r), wf[j]));
+      st_vec<T, V>(row + i, q);
+      if (store) st_vec<T, V>(xn + (size_t)t * d + i, q);
     }
     __syncthreads();
     if (logits != nullptr) {
@@ -99,10 +106,11 @@ __global__ void __launch_bounds__(256) rmsnorm_router_kernel(const T* __restrict
         const T* wr = w_router + (size_t)e * d;
         float s = 0.f;
         for (int i = lane_id() * V; i < d; i += 32 * V) {
-          float wf[V];
-          load_vec<T, V>(wr + i, wf);
+          float xf[V], wf[V];
+          vec_to_f32(ld_vec<T, V>(row + i), xf);
+          vec_to_f32(ld_vec<T, V>(wr + i), wf);
 #pragma unroll
-          for (int j = 0; j < V; ++j) s = __fmaf_rn(row[i + j], wf[j], s);
+          for (int j = 0; j < V; ++j) s = __fmaf_rn(xf[j], wf[j], s);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -214,7 +222,7 @@ namespace moe_host {
 template <typename T, int V>
 static moe_status launch_rr(const void* h, const void* norm_w, const void* w_router, void* xn, float* logits, int n,
                             int d, int e, float eps, cudaStream_t s) {
-  const size_t smem = sizeof(float) * (size_t)d;
+  const size_t smem = sizeof(T) * (size_t)d;
   auto kern = moe::rmsnorm_router_kernel<T, V>;
   if (smem > 48 * 1024) {
     static bool done[64] = {};
