@@ -234,6 +234,14 @@ moe_status moe_check_device_error(void* ws, size_t ws_bytes, void* stream, int32
  * the first unsuccessful poll). */
 moe_status moe_set_wait_timeout_ns(int64_t ns);
 
+/* Tile shape of the bf16 grouped expert GEMMs for launches after this call
+ * (process-wide): 0 = choose per launch (the default: SM-pair 256-row tiles
+ * for the down projection and the router when the groups average at least
+ * 512 rows, single-SM 128-row tiles otherwise),
+ * 1 = single-SM tiles, 2 = SM-pair tiles.  Results are the same up to
+ * floating-point summation order; this is a performance control. */
+moe_status moe_set_gemm_tiling(int32_t mode);
+
 /* Launch one block that waits on a workspace flag that nothing sets, with
  * the current wait limit: it must give up and record MOE_ERR_DEVICE_TIMEOUT.
  * Exercises the timeout path without faulting or hanging the GPU. */

@@ -32,7 +32,7 @@ MOE_F32, MOE_BF16 = 0, 1
 ENTRY_POINTS = (
     "moe_status_string", "moe_version", "moe_workspace_size", "moe_workspace_init", "moe_route",
     "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_bias_update",
-    "moe_check_device_error", "moe_set_wait_timeout_ns", "moe_selftest_wait_timeout",
+    "moe_check_device_error", "moe_set_wait_timeout_ns", "moe_set_gemm_tiling", "moe_selftest_wait_timeout",
 )
 
 
@@ -85,6 +85,7 @@ def _load():
         "moe_bias_update": (I32, [I32, P, F, F, P, P]),
         "moe_check_device_error": (I32, [P, SZ, P, P]),
         "moe_set_wait_timeout_ns": (I32, [I64]),
+        "moe_set_gemm_tiling": (I32, [I32]),
         "moe_selftest_wait_timeout": (I32, [P, SZ, P]),
     }
     for name, (res, args) in sig.items():
@@ -264,6 +265,11 @@ def moe_check_device_error(ws, stream=None):
 
 def moe_set_wait_timeout_ns(ns: int):
     _check(_lib.moe_set_wait_timeout_ns(int(ns)), "moe_set_wait_timeout_ns")
+
+
+def moe_set_gemm_tiling(mode: int):
+    """0 = automatic, 1 = single-SM 128-row tiles, 2 = SM-pair 256-row tiles."""
+    _check(_lib.moe_set_gemm_tiling(int(mode)), "moe_set_gemm_tiling")
 
 
 def moe_selftest_wait_timeout(ws, stream=None):

@@ -6,6 +6,7 @@
 
 #include "moe_common.cuh"
 #include "moe_kernels.h"
+#include "tcgen05.cuh"
 
 namespace moe_host {
 
@@ -331,6 +332,12 @@ moe_status moe_check_device_error(void* ws, size_t ws_bytes, void* stream, int32
 moe_status moe_set_wait_timeout_ns(int64_t ns) {
   if (ns < 0) return MOE_ERR_INVALID_ARG;
   g_wait_ns = (uint64_t)ns;
+  return MOE_OK;
+}
+
+moe_status moe_set_gemm_tiling(int32_t mode) {
+  if (mode < 0 || mode > 2) return MOE_ERR_INVALID_ARG;
+  set_tc_pairing(mode);
   return MOE_OK;
 }
 

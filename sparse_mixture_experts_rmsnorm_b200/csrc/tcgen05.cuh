@@ -1,0 +1,240 @@
+// tcgen05 / TMA building blocks shared by the grouped GEMM kernels
+// (single-SM tiles in gemm_tc.cu, SM-pair tiles in gemm_tc2.cu): argument
+// block, PTX wrappers, shared-memory and instruction descriptors, the TMEM
+// load, the work schedule and the epilogue of one accumulator row.
+#pragma once
+
+#include <cuda.h>
+
+#include "moe_common.cuh"
+#include "moe_kernels.h"
+
+namespace moe {
+
+constexpr int TC_BK = 64;  // k-block: 128 bytes of bf16, one 128-byte swizzle row
+constexpr int TC_MAX_GROUPS = 1024;
+constexpr uint32_t TC_TMEM_COLS = 512;
+
+// wait sites (word 3 of the error record)
+enum { SITE_EMPTY = 1, SITE_FULL = 2, SITE_TMEM_EMPTY = 3, SITE_TMEM_FULL = 4, SITE_DRAIN = 5 };
+
+struct TcArgs {
+  const int32_t* offsets;  // [G+1] device, or nullptr: one group of max_rows rows
+  int groups;
+  int max_rows;
+  int nout;        // output columns per group (H, d or E)
+  int K;
+  int n_tiles;     // n-tiles per group
+  int out_cols;    // output columns per tile: 128 (SwiGLU) or 256
+  void* C;
+  int ldc;
+  int32_t* hdr;
+  uint64_t wait_ns;
+};
+
+// ---- PTX wrappers -----------------------------------------------------------
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (bf16 in, fp32 accumulate).
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                       uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major tile written by TMA with the
+// 128-byte swizzle: rows of 128 bytes, 8-row groups 1024 bytes apart.
+// Fields: start address >> 4 (bits 0-13), leading byte offset (unused by
+// swizzled K-major layouts, 1), stride byte offset 1024 >> 4 (bits 32-45),
+// descriptor version 1 (bits 46-47), swizzle mode 2 = 128 B (bits 61-63).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulator (bits 4-5 = 1), A and
+// B bf16 (bits 7-9 = 1, 10-12 = 1), both K-major, N >> 3 at bit 17,
+// M >> 4 at bit 24.
+constexpr uint32_t tc_idesc(int m, int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+#define MOE_TMEM_LD32(taddr, r)                                                                                   \
+  asm volatile(                                                                                                   \
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, " \
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"              \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),           \
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),     \
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),   \
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])    \
+      : "r"(taddr))
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float silu_tc(float z) { return __fdiv_rn(z, __fadd_rn(1.f, expf(-z))); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);  // .x = lo (lower address), .y = hi
+  return *reinterpret_cast<uint32_t*>(&p);
+}
+
+// Store 32 consecutive columns [col, col + 32) of one output row as bf16,
+// masked to col < nout; 16-byte stores when the row allows them.
+__device__ __forceinline__ void store_row32_bf16(bf16* out, int col, int nout, bool vec_ok, const float (&v)[32]) {
+  if (vec_ok && col + 32 <= nout) {
+    uint4* dst = reinterpret_cast<uint4*>(out + col);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      dst[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]), pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                          pack_bf16x2(v[8 * q + 4], v[8 * q + 5]), pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (col + i < nout) out[col + i] = __float2bfloat16_rn(v[i]);
+  }
+}
+
+// ---- tile schedule -----------------------------------------------------------
+// Tiles of BM rows; a group of r rows has ceil(r / BM) m-tiles and n_tiles
+// n-tiles; prefix[g] is the first tile of group g.
+struct Tile {
+  int group, row0, row_end, n0;
+};
+
+template <int BM>
+__device__ __forceinline__ void build_prefix(const int* offs, int* prefix, int groups, int n_tiles) {
+  // one warp: exclusive scan of the tile counts
+  const int lane = lane_id();
+  int carry = 0;
+  for (int base = 0; base < groups; base += 32) {
+    const int g = base + lane;
+    const int v = (g < groups) ? ((offs[g + 1] - offs[g] + BM - 1) / BM) * n_tiles : 0;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (g < groups) prefix[g] = carry + x - v;
+    carry += __shfl_sync(0xffffffffu, x, 31);
+  }
+  if (lane == 0) prefix[groups] = carry;
+}
+
+template <int BM>
+__device__ __forceinline__ Tile decode_tile(int t, const int* prefix, const int* offs, int groups, int out_cols) {
+  int lo = 0, hi = groups - 1;  // last g with prefix[g] <= t
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if (prefix[mid] <= t) lo = mid;
+    else hi = mid - 1;
+  }
+  const int g = lo;
+  const int rows = offs[g + 1] - offs[g];
+  const int mt = (rows + BM - 1) / BM;
+  const int local = t - prefix[g];
+  Tile tl;
+  tl.group = g;
+  tl.row0 = offs[g] + (local % mt) * BM;
+  tl.row_end = offs[g + 1];
+  tl.n0 = (local / mt) * out_cols;
+  return tl;
+}
+
+// ---- epilogue of one accumulator row -----------------------------------------
+// The calling thread owns TMEM lane `tbase` (row `row` of the output) and
+// drains 256 accumulator columns starting at tbase's column:
+//   EPI_SWIGLU: columns c and 128 + c are the gate and up halves of hidden
+//               unit n0 + c; writes silu(gate) * up for 128 units;
+//   EPI_STORE / EPI_F32: writes the 256 columns n0 .. n0 + 255.
+// Stores are masked to row_ok and to columns < nout.  All 32 lanes of the
+// warp must call it (tcgen05.ld is warp-wide).
+template <int EPI>
+__device__ __forceinline__ void epilogue_row(const TcArgs& args, uint32_t tbase, int row, bool row_ok, int n0) {
+  if (EPI == moe_host::EPI_SWIGLU) {
+    bf16* out = reinterpret_cast<bf16*>(args.C) + (size_t)row * args.ldc;
+#pragma unroll 1
+    for (int c = 0; c < 128; c += 32) {
+      uint32_t g[32], u[32];
+      MOE_TMEM_LD32(tbase + c, g);
+      MOE_TMEM_LD32(tbase + 128 + c, u);
+      tmem_wait_ld();
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(silu_tc(__uint_as_float(g[i])), __uint_as_float(u[i]));
+      if (row_ok) store_row32_bf16(out, n0 + c, args.nout, (args.ldc & 7) == 0, v);
+    }
+  } else {
+#pragma unroll 1
+    for (int c = 0; c < 256; c += 32) {
+      uint32_t a[32];
+      MOE_TMEM_LD32(tbase + c, a);
+      tmem_wait_ld();
+      const int col = n0 + c;
+      if (!row_ok) continue;
+      if (EPI == moe_host::EPI_F32) {
+        float* out = reinterpret_cast<float*>(args.C) + (size_t)row * args.ldc;
+        if (col + 32 <= args.nout && (args.ldc & 3) == 0) {
+          uint4* dst = reinterpret_cast<uint4*>(out + col);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) dst[q] = make_uint4(a[4 * q], a[4 * q + 1], a[4 * q + 2], a[4 * q + 3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (col + i < args.nout) out[col + i] = __uint_as_float(a[i]);
+        }
+      } else {
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(a[i]);
+        store_row32_bf16(reinterpret_cast<bf16*>(args.C) + (size_t)row * args.ldc, col, args.nout,
+                         (args.ldc & 7) == 0, v);
+      }
+    }
+  }
+}
+
+}  // namespace moe
+
+namespace moe_host {
+// 2-D bf16 tensor map over a row-major [rows][k] matrix: box 128 rows x 64
+// columns, 128-byte swizzle, zero fill outside the matrix.
+bool make_tc_map(CUtensorMap* m, const void* base, int64_t rows, int k);
+
+// The SM-pair kernel (gemm_tc2.cu) on maps and arguments prepared by
+// launch_gemm_tc; groups_bound = groups when offsets are given, else 0.
+moe_status launch_gemm_tc2(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
+                           const moe::TcArgs& args, int64_t max_rows, int groups_bound, cudaStream_t s);
+
+// 0: choose per launch (SM pairs for the store / fp32 epilogues when the
+//    groups average >= 512 rows);
+// 1: single-SM tiles only; 2: SM-pair tiles only.
+void set_tc_pairing(int mode);
+int tc_pairing();
+}  // namespace moe_host

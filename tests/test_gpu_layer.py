@@ -194,21 +194,47 @@ def _ffn_case(torch, groups_rows, d, H, seed, with_offsets=True):
     return got[:R], ref
 
 
+@pytest.fixture
+def gemm_tiling():
+    import sparse_mixture_experts_rmsnorm_b200 as moe
+
+    def set_mode(mode):
+        moe.moe_set_gemm_tiling(mode)
+    yield set_mode
+    moe.moe_set_gemm_tiling(0)
+
+
+@pytest.mark.parametrize("mode", [1, 2])  # single-SM 128-row tiles, SM-pair 256-row tiles
 @pytest.mark.parametrize("rows,d,H", [
     ([0, 130, 77, 1, 256], 192, 200),      # ragged groups, empty group, partial tiles, 3 k-blocks
     ([300], 4096, 512),                    # one group, many k-blocks
     ([5, 0, 0, 129, 64], 520, 1032),       # K and N not multiples of the tile
+    ([700, 1300, 0, 513, 256], 256, 384),  # groups spanning several SM-pair tiles
 ])
-def test_expert_ffn_tc_matches_oracle(torch_cuda, rows, d, H):
+def test_expert_ffn_tc_matches_oracle(torch_cuda, gemm_tiling, rows, d, H, mode):
+    gemm_tiling(mode)
     got, ref = _ffn_case(torch_cuda, rows, d, H, seed=len(rows) + d)
     err = bf16_rel_rms_err(got, ref)
-    print(f"expert FFN {rows} d={d} H={H}: beyond-storage max err/rms {err:.3e}, raw {rel_rms_err(got, ref):.3e}")
+    print(f"expert FFN tiling {mode} {rows} d={d} H={H}: beyond-storage max err/rms {err:.3e}, "
+          f"raw {rel_rms_err(got, ref):.3e}")
     assert err <= BF16_REL_RMS, err
 
 
-def test_expert_ffn_tc_single_group_smaller_than_a_tile(torch_cuda):
+@pytest.mark.parametrize("mode", [1, 2])
+def test_expert_ffn_tc_single_group_smaller_than_a_tile(torch_cuda, gemm_tiling, mode):
+    gemm_tiling(mode)
     got, ref = _ffn_case(torch_cuda, [64], 256, 256, seed=5, with_offsets=False)
     assert bf16_rel_rms_err(got, ref) <= BF16_REL_RMS
+
+
+def test_both_tilings_agree_closely(torch_cuda, gemm_tiling):
+    # same products, summation order aside
+    gemm_tiling(1)
+    a, ref = _ffn_case(torch_cuda, [600, 900], 512, 640, seed=9)
+    gemm_tiling(2)
+    b, _ = _ffn_case(torch_cuda, [600, 900], 512, 640, seed=9)
+    assert rel_rms_err(a, b) <= 2e-2
+    assert bf16_rel_rms_err(b, ref) <= BF16_REL_RMS
 
 
 # ----------------------------------------------------------------- router on the tensor cores
