@@ -54,7 +54,7 @@ import numpy as np
 __all__ = [
     "round_to", "rmsnorm", "router_scores", "select_topk", "gates_from_scores",
     "expert_counts", "capacity_limit", "permute", "silu", "swiglu_expert",
-    "combine", "layer_forward", "bias_update",
+    "combine", "layer_forward", "bias_update", "balancing_loop",
 ]
 
 
@@ -242,6 +242,28 @@ def bias_update(bias, counts, target: float, gamma: float) -> np.ndarray:
     c = np.asarray(counts).astype(np.float32)
     s = np.sign(np.float32(target) - c).astype(np.float32)
     return (b + s * np.float32(gamma)).astype(np.float32)
+
+
+def balancing_loop(scores, bias0, k: int, target: float, gamma: float, iterations: int):
+    """Repeated aux-loss-free balancing on fixed router scores.
+
+    [LESSON] "Step 2: run 100 tokens through the router": route every token,
+    count each expert's load, move every bias by -gamma (over target) or
+    +gamma (under target), repeat.  Each iteration selects on the current
+    bias (select_topk), counts before any capacity cut (expert_counts) and
+    applies bias_update.  Returns (counts [iterations, E], biases
+    [iterations + 1, E] fp32), biases[0] = bias0.
+    """
+    bias = np.asarray(bias0, dtype=np.float32).copy()
+    n_experts = np.asarray(scores).shape[1]
+    counts, biases = [], [bias.copy()]
+    for _ in range(iterations):
+        idx, _ = select_topk(scores, bias, k)
+        c = expert_counts(idx, n_experts)
+        bias = bias_update(bias, c, target, gamma)
+        counts.append(c)
+        biases.append(bias.copy())
+    return np.array(counts), np.array(biases)
 
 
 # ----------------------------------------------------------------------------

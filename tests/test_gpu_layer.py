@@ -314,3 +314,33 @@ def test_small_bf16_layer_every_output(torch_cuda, over):
     if cfg.d_ff_shared == 0 and dropped_all.size:
         np.testing.assert_array_equal(g["out"][dropped_all], ref["h"][dropped_all] if "h" in ref else
                                       mi.host_tensor(cfg, "h")[dropped_all])
+
+
+# ----------------------------------------------------------------- the forward pass as a CUDA graph
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "dsv3_decode_bf16"])
+def test_layer_forward_replays_from_a_cuda_graph(torch_cuda, name):
+    # moe_layer_forward enqueues work on one stream with no host synchronisation,
+    # so a captured graph replays the identical computation
+    torch = torch_cuda
+    import sparse_mixture_experts_rmsnorm_b200 as moe
+    cfg = mi.CONFIGS[name]
+    lc = lib_config(cfg)
+    dev = mi.device_tensors(cfg)
+    w = {n: dev[n] for n in ("norm_w", "w_router", "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down")
+         if n in dev}
+    ws = moe.workspace(lc)
+    eager = torch.empty_like(dev["h"])
+    moe.moe_layer_forward(lc, w, dev["h"], dev["bias"], eager, ws)  # also warms every kernel up
+    torch.cuda.synchronize()
+    out = torch.zeros_like(dev["h"])
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        moe.moe_layer_forward(lc, w, dev["h"], dev["bias"], out, ws)
+    for _ in range(2):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager)
+    st, info = moe.moe_check_device_error(ws)
+    assert st == 0, info

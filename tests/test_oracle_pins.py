@@ -311,3 +311,39 @@ def test_stress_recipe_skews_top1_to_expert3_and_bias_signs():
     g = np.float32(cfg.gamma)
     assert nb[3] == -g and all(nb[e] == g for e in range(8) if e != 3)
     assert oracle.capacity_limit(cfg.capacity_factor, cfg.n_tokens, cfg.top_k, cfg.n_experts) == 1280
+
+
+# ---------------------------------------------------------------- iterated balancing (lesson, Step 2)
+
+def test_balancing_loop_two_experts_hand_derived_trajectory():
+    # Every token scores (0.625, 0.375); gamma = 2^-7, so all sums are exact.
+    # Expert 0 takes all tokens while 0.625 - n*g > 0.375 + n*g, i.e. for
+    # n = 0..15; at n = 16 the keys tie (0.5, 0.5) and the lower index keeps
+    # them, so the bias moves once more; at n = 17 expert 1 wins, the biases
+    # step back to n = 16 and the pair oscillates: counts alternate from then on.
+    n_tok, g = 10, 2.0 ** -7
+    scores = np.tile([0.625, 0.375], (n_tok, 1))
+    counts, biases = oracle.balancing_loop(scores, [0.0, 0.0], 1, n_tok / 2, g, 22)
+    assert counts[:17, 0].tolist() == [n_tok] * 17
+    assert counts[17:, 0].tolist() == [0, n_tok, 0, n_tok, 0]
+    assert biases[17].tolist() == [-17 * g, 17 * g]
+    assert biases[18].tolist() == [-16 * g, 16 * g]
+    assert biases[22].tolist() == [-16 * g, 16 * g]
+    assert counts.sum(axis=1).tolist() == [n_tok] * 22
+
+
+def test_balancing_loop_reduces_imbalance():
+    # [LESSON] "Step 2": with the bias loop, skewed usage moves to a near
+    # uniform one within some tens of iterations.  Router logits with
+    # per-expert offsets 0 .. 2 start about 2.3x over the mean load.
+    r = np.random.default_rng(3)
+    xn = r.standard_normal((1024, 32))
+    logits = xn @ (r.standard_normal((8, 32)) / np.sqrt(32)).T + np.linspace(0, 2, 8)
+    ex = np.exp(logits - logits.max(1, keepdims=True))
+    scores = ex / ex.sum(1, keepdims=True)
+    counts, biases = oracle.balancing_loop(scores, np.zeros(8), 2, 1024 * 2 / 8, 5e-3, 50)
+    ratio = counts.max(axis=1) / counts.mean(axis=1)
+    assert ratio[0] > 2.0 and ratio[-10:].max() < 1.2 and ratio[-1] < 1.1
+    assert np.all(counts.sum(axis=1) == 2048)
+    # the most loaded expert at the start ends with the lowest bias
+    assert np.argmin(biases[-1]) == np.argmax(counts[0])
