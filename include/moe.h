@@ -137,6 +137,20 @@ moe_status moe_route(const moe_config* cfg, const void* h, const void* norm_w, c
                      const float* bias, void* xn, float* scores, int32_t* topk_idx, float* topk_gate,
                      int32_t* counts, void* ws, size_t ws_bytes, void* stream);
 
+/* Hash routing in place of steps a2-a3 (the lesson's exercise of a hash
+ * router that routes without learning: "Mixture of Experts (MoE)" lesson,
+ * "Exercises").  Computes xn = RMSNorm(h) as moe_route does, then for token
+ * t with id x = token_ids[t] (token_ids NULL: x = t) chooses experts
+ *   e_j = (splitmix64(x) + j) mod E,  j = 0 .. k-1,
+ * splitmix64 being the SplitMix64 output function (Steele, Lea and Flood,
+ * 2014), with every gate 1/k.  The result feeds moe_permute, moe_expert_ffn
+ * and moe_combine unchanged.
+ *   token_ids [N] int64 device or NULL; xn, topk_idx, topk_gate, counts: out,
+ *   as in moe_route.  Errors as moe_route. */
+moe_status moe_route_hash(const moe_config* cfg, const void* h, const void* norm_w, const int64_t* token_ids,
+                          void* xn, int32_t* topk_idx, float* topk_gate, int32_t* counts, void* ws, size_t ws_bytes,
+                          void* stream);
+
 /* Step a4-a5: per-expert counting sort of the N*k routing slots, capacity and
  * gather.  Glossary "Load balancing and expert capacity" (tokens per expert,
  * overflow continues on the residual); lesson "The load-balancing problem"

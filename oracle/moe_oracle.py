@@ -54,7 +54,7 @@ import numpy as np
 __all__ = [
     "round_to", "rmsnorm", "router_scores", "select_topk", "gates_from_scores",
     "expert_counts", "capacity_limit", "permute", "silu", "swiglu_expert",
-    "combine", "layer_forward", "bias_update", "balancing_loop",
+    "combine", "layer_forward", "bias_update", "balancing_loop", "splitmix64", "hash_route",
 ]
 
 
@@ -264,6 +264,36 @@ def balancing_loop(scores, bias0, k: int, target: float, gamma: float, iteration
         counts.append(c)
         biases.append(bias.copy())
     return np.array(counts), np.array(biases)
+
+
+# ----------------------------------------------------------------------------
+# Hash router ([LESSON] "Exercises": a hash router that routes tokens without
+# learning).  Reading taken: the expert of choice j is (h(id) + j) mod E, with
+# h the SplitMix64 output function (Steele, Lea, Flood 2014) applied to the
+# token id, and every chosen expert gets gate 1/k.
+# ----------------------------------------------------------------------------
+
+_M64 = (1 << 64) - 1
+
+
+def splitmix64(x: int) -> int:
+    """One SplitMix64 output for state x: mix(x + golden gamma), 64-bit wrap."""
+    z = (x + 0x9E3779B97F4A7C15) & _M64
+    z = ((z ^ (z >> 30)) * 0xBF58476D1CE4E5B9) & _M64
+    z = ((z ^ (z >> 27)) * 0x94D049BB133111EB) & _M64
+    return z ^ (z >> 31)
+
+
+def hash_route(token_ids, n_experts: int, k: int):
+    """Returns (idx [N, k] int64, gates [N, k] float32)."""
+    ids = [int(t) & _M64 for t in np.asarray(token_ids).ravel().tolist()]
+    idx = np.empty((len(ids), k), dtype=np.int64)
+    for t, tid in enumerate(ids):
+        e0 = splitmix64(tid) % n_experts
+        for j in range(k):
+            idx[t, j] = (e0 + j) % n_experts
+    gates = np.full((len(ids), k), np.float32(1.0) / np.float32(k), dtype=np.float32)
+    return idx, gates
 
 
 # ----------------------------------------------------------------------------

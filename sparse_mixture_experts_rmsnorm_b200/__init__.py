@@ -30,7 +30,7 @@ MOE_F32, MOE_BF16 = 0, 1
 
 # Every entry point declared in include/moe.h, in declaration order.
 ENTRY_POINTS = (
-    "moe_status_string", "moe_version", "moe_workspace_size", "moe_workspace_init", "moe_route",
+    "moe_status_string", "moe_version", "moe_workspace_size", "moe_workspace_init", "moe_route", "moe_route_hash",
     "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_bias_update",
     "moe_check_device_error", "moe_set_wait_timeout_ns", "moe_set_gemm_tiling", "moe_selftest_wait_timeout",
 )
@@ -76,6 +76,7 @@ def _load():
         "moe_workspace_size": (SZ, [cfgp]),
         "moe_workspace_init": (I32, [P, SZ, P]),
         "moe_route": (I32, [cfgp, P, P, P, P, P, P, P, P, P, P, SZ, P]),
+        "moe_route_hash": (I32, [cfgp, P, P, P, P, P, P, P, P, SZ, P]),
         "moe_permute": (I32, [cfgp, P, P, P, P, P, P, P, SZ, P]),
         "moe_permute_noalloc": (I32, [cfgp, P, P, P, P, P, P, P]),
         "moe_expert_ffn": (I32, [cfgp, I32, P, I32, P, P, P, P, I32, P, P, SZ, P]),
@@ -194,6 +195,14 @@ def moe_route(cfg: Config, h, norm_w, w_router, bias, xn, scores, topk_idx, topk
     _check(_lib.moe_route(ctypes.byref(cfg.c()), _ptr(h), _ptr(norm_w), _ptr(w_router), _ptr(bias), _ptr(xn),
                           _ptr(scores), _ptr(topk_idx), _ptr(topk_gate), _ptr(counts), _ptr(ws), ws.numel(),
                           _stream(stream)), "moe_route")
+
+
+def moe_route_hash(cfg: Config, h, norm_w, token_ids, xn, topk_idx, topk_gate, counts, ws, stream=None):
+    """RMSNorm, then routing by a SplitMix64 hash of each token id (token_ids: int64
+    tensor or None for the token's position); gates 1/k."""
+    _check(_lib.moe_route_hash(ctypes.byref(cfg.c()), _ptr(h), _ptr(norm_w), _ptr(token_ids), _ptr(xn),
+                               _ptr(topk_idx), _ptr(topk_gate), _ptr(counts), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_route_hash")
 
 
 def moe_permute(cfg: Config, topk_idx, xn, offsets, slot_row, row_token, x_perm, ws, stream=None):

@@ -212,6 +212,19 @@ moe_status moe_route(const moe_config* cfg, const void* h, const void* norm_w, c
                     (cudaStream_t)stream);
 }
 
+moe_status moe_route_hash(const moe_config* cfg, const void* h, const void* norm_w, const int64_t* token_ids,
+                          void* xn, int32_t* topk_idx, float* topk_gate, int32_t* counts, void* ws, size_t ws_bytes,
+                          void* stream) {
+  MOE_TRY(check_common(cfg, ws, ws_bytes));
+  if (cfg->n_tokens > 0 && (!h || !norm_w || !xn || !topk_idx || !topk_gate)) return MOE_ERR_INVALID_ARG;
+  if (!counts) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cfg->n_tokens > 0)
+    MOE_TRY(launch_rmsnorm_router(cfg->dtype, h, norm_w, nullptr, xn, nullptr, cfg->n_tokens, cfg->d_model,
+                                  cfg->n_experts, cfg->rms_eps, s));
+  return launch_hash_route(token_ids, topk_idx, topk_gate, counts, cfg->n_tokens, cfg->n_experts, cfg->top_k, s);
+}
+
 moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* xn, int32_t* offsets,
                        int32_t* slot_row, int32_t* row_token, void* x_perm, void* ws, size_t ws_bytes,
                        void* stream) {

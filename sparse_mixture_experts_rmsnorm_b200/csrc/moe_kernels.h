@@ -26,6 +26,11 @@ moe_status launch_rmsnorm_router(int dtype, const void* h, const void* norm_w, c
 moe_status launch_topk(const float* logits, const float* bias, float* scores, int32_t* topk_idx,
                        float* topk_gate, int32_t* counts, int n, int e, int k, cudaStream_t s);
 
+// Hash router: choice j of token t is (splitmix64(id) + j) mod E, id =
+// token_ids[t] (or t when token_ids is null), gates 1/k; counts zeroed first.
+moe_status launch_hash_route(const int64_t* token_ids, int32_t* topk_idx, float* topk_gate, int32_t* counts, int n,
+                             int e, int k, cudaStream_t s);
+
 // a4: stable counting sort of the N*k slots by expert with optional capacity.
 //   hist: workspace of permute_hist_ints(n*k, e) int32.
 size_t permute_hist_ints(int64_t slots, int e);

@@ -215,9 +215,57 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     if (hist[e]) atomicAdd(&counts[e], hist[e]);
 }
 
+// ---------------------------------------------------------------------------
+// Hash router ("Mixture of Experts (MoE)" lesson, "Exercises": route tokens
+// with a hash instead of a learned router).  Choice j of a token with id x is
+// (h(x) + j) mod E, h the SplitMix64 output function (Steele, Lea and Flood,
+// "Fast splittable pseudorandom number generators", 2014); every gate 1/k.
+// One thread per token; counts through a per-block shared histogram.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t splitmix64_mix(uint64_t x) {
+  uint64_t z = x + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+__global__ void __launch_bounds__(256) hash_route_kernel(const int64_t* __restrict__ token_ids, int n, int E, int k,
+                                                         int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate,
+                                                         int32_t* __restrict__ counts) {
+  extern __shared__ int32_t hist[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const float g = __fdiv_rn(1.f, (float)k);
+  for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < n; t += gridDim.x * blockDim.x) {
+    const uint64_t id = token_ids ? (uint64_t)token_ids[t] : (uint64_t)t;
+    const int e0 = (int)(splitmix64_mix(id) % (uint64_t)E);
+    for (int j = 0; j < k; ++j) {
+      int e = e0 + j;
+      if (e >= E) e -= E;
+      topk_idx[(size_t)t * k + j] = e;
+      topk_gate[(size_t)t * k + j] = g;
+      atomicAdd(&hist[e], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (hist[e]) atomicAdd(&counts[e], hist[e]);
+}
+
 }  // namespace moe
 
 namespace moe_host {
+
+moe_status launch_hash_route(const int64_t* token_ids, int32_t* topk_idx, float* topk_gate, int32_t* counts, int n,
+                             int e, int k, cudaStream_t s) {
+  if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * e, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (n == 0) return MOE_OK;
+  int blocks = (n + 255) / 256;
+  if (blocks > sm_count() * 4) blocks = sm_count() * 4;
+  moe::hash_route_kernel<<<blocks, 256, sizeof(int32_t) * e, s>>>(token_ids, n, e, k, topk_idx, topk_gate, counts);
+  return launch_status();
+}
+
 
 template <typename T, int V>
 static moe_status launch_rr(const void* h, const void* norm_w, const void* w_router, void* xn, float* logits, int n,

@@ -347,3 +347,27 @@ def test_balancing_loop_reduces_imbalance():
     assert np.all(counts.sum(axis=1) == 2048)
     # the most loaded expert at the start ends with the lowest bias
     assert np.argmin(biases[-1]) == np.argmax(counts[0])
+
+
+# ---------------------------------------------------------------- hash router (lesson exercise)
+
+def test_splitmix64_published_first_output():
+    # the first SplitMix64 output from state 0 (Vigna's splitmix64.c)
+    assert oracle.splitmix64(0) == 0xE220A8397B1DCDAF
+
+
+def test_hash_route_properties():
+    E, k = 16, 3
+    ids = np.arange(20000)
+    idx, gates = oracle.hash_route(ids, E, k)
+    assert idx[0, 0] == 0xE220A8397B1DCDAF % E
+    # k distinct, consecutive (mod E) experts; gates 1/k in fp32
+    assert np.all((idx[:, 1] - idx[:, 0]) % E == 1) and np.all((idx[:, 2] - idx[:, 0]) % E == 2)
+    np.testing.assert_array_equal(gates, np.float32(1 / 3))
+    # the first choice is close to uniform over the experts (chi-square, 15 dof, p ~ 1e-4 bound)
+    c = np.bincount(idx[:, 0], minlength=E)
+    chi2 = ((c - len(ids) / E) ** 2 / (len(ids) / E)).sum()
+    assert chi2 < 45
+    # the same id always routes the same way
+    again, _ = oracle.hash_route(ids[::-1], E, k)
+    np.testing.assert_array_equal(again[::-1], idx)
