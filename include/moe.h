@@ -113,7 +113,10 @@ const char* moe_version(void);
  * error word), xn, the routing buffers that moe_routing leaves NULL, router
  * logits, permutation histograms, the expert-sorted rows x_perm [R][d],
  * activations [max(R*H, N*Hs)] and expert outputs y_perm [R][d], y_shared
- * [N][d], where R = N*k, or min(N*k, E*cap) with a capacity. */
+ * [N][d], where R = N*k, or min(N*k, E*cap) with a capacity.  When the
+ * shared expert is as wide as the routed ones (bf16, Hs == H) it runs as one
+ * more group of the routed expert GEMMs: x_perm, act and y_perm then hold
+ * R + N rows and there is no separate y_shared. */
 size_t moe_workspace_size(const moe_config* cfg);
 
 /* Zero the workspace header (the device error word).  Call once after

@@ -20,13 +20,15 @@ namespace moe {
 //   out = round(acc).
 // A token whose slots are all dropped (and no shared expert) returns h exactly.
 // VEC consecutive elements per thread (VEC * sizeof(T) = 16 bytes when aligned).
-template <typename T, int VEC>
+template <typename T, int VEC, int KC>
 __global__ void __launch_bounds__(128) combine_kernel(const T* __restrict__ h, const T* __restrict__ y_perm,
                                                       const int32_t* __restrict__ slot_row,
                                                       const float* __restrict__ gates,
                                                       const T* __restrict__ y_shared, T* out, int n, int d,
-                                                      int k) {
+                                                      int k, const int32_t* __restrict__ shared_offsets, int E) {
   __shared__ int32_t rows[32];
+  // the folded shared expert: its rows follow the routed rows of y_perm
+  if (shared_offsets != nullptr) y_shared = y_perm + (size_t)shared_offsets[E] * d;
   __shared__ float g[32];
   for (int t = blockIdx.x; t < n; t += gridDim.x) {
     if (threadIdx.x < k) {
@@ -45,18 +47,27 @@ __global__ void __launch_bounds__(128) combine_kernel(const T* __restrict__ h, c
       }
 #pragma unroll
       for (int i = 0; i < VEC; ++i) acc[i] = to_f32(tmp[i]);
-      for (int j = 0; j < k; ++j) {
-        const int r = rows[j];
-        if (r < 0) continue;
-        const float gj = g[j];
-        const T* yr = y_perm + (size_t)r * d + c;
-        if (VEC > 1) {
-          *reinterpret_cast<uint4*>(tmp) = *reinterpret_cast<const uint4*>(yr);
-        } else {
-          tmp[0] = yr[0];
+      // up to KC slot rows in flight per thread, summed in rank order
+      for (int j0 = 0; j0 < k; j0 += KC) {
+        T yv[KC][VEC];
+#pragma unroll
+        for (int jj = 0; jj < KC; ++jj) {
+          const int j = j0 + jj;
+          if (j < k && rows[j] >= 0) {
+            const T* yr = y_perm + (size_t)rows[j] * d + c;
+            if (VEC > 1) *reinterpret_cast<uint4*>(yv[jj]) = *reinterpret_cast<const uint4*>(yr);
+            else yv[jj][0] = yr[0];
+          }
         }
 #pragma unroll
-        for (int i = 0; i < VEC; ++i) acc[i] = __fmaf_rn(gj, to_f32(tmp[i]), acc[i]);
+        for (int jj = 0; jj < KC; ++jj) {
+          const int j = j0 + jj;
+          if (j < k && rows[j] >= 0) {
+            const float gj = g[j];
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) acc[i] = __fmaf_rn(gj, to_f32(yv[jj][i]), acc[i]);
+          }
+        }
       }
       if (y_shared != nullptr) {
         if (VEC > 1) {
@@ -93,29 +104,35 @@ __global__ void bias_update_kernel(int E, const int32_t* __restrict__ counts, fl
 
 namespace moe_host {
 
+template <typename T, int VEC>
+static void launch_combine_t(const void* h, const void* y_perm, const int32_t* slot_row, const float* topk_gate,
+                             const void* y_shared, void* out, int n, int d, int k, const int32_t* shared_offsets,
+                             int e, int grid, cudaStream_t s) {
+#define MOE_COMBINE(KC)                                                                                    \
+  moe::combine_kernel<T, VEC, KC><<<grid, 128, 0, s>>>((const T*)h, (const T*)y_perm, slot_row, topk_gate, \
+                                                       (const T*)y_shared, (T*)out, n, d, k, shared_offsets, e)
+  if (k <= 2) MOE_COMBINE(2);
+  else if (k <= 4) MOE_COMBINE(4);
+  else MOE_COMBINE(8);
+#undef MOE_COMBINE
+}
+
 moe_status launch_combine(int dtype, const void* h, const void* y_perm, const int32_t* slot_row,
                           const float* topk_gate, const void* y_shared, void* out, int n, int d, int k,
-                          cudaStream_t s) {
+                          cudaStream_t s, const int32_t* shared_offsets, int e) {
   if (n == 0) return MOE_OK;
   int grid = n < sm_count() * 16 ? n : sm_count() * 16;
   const uintptr_t addr = (uintptr_t)h | (uintptr_t)y_perm | (uintptr_t)y_shared | (uintptr_t)out;
   if (dtype == MOE_BF16) {
-    typedef moe::bf16 T;
     if (d % 8 == 0 && addr % 16 == 0)
-      moe::combine_kernel<T, 8><<<grid, 128, 0, s>>>((const T*)h, (const T*)y_perm, slot_row, topk_gate,
-                                                     (const T*)y_shared, (T*)out, n, d, k);
+      launch_combine_t<moe::bf16, 8>(h, y_perm, slot_row, topk_gate, y_shared, out, n, d, k, shared_offsets, e, grid, s);
     else
-      moe::combine_kernel<T, 1><<<grid, 128, 0, s>>>((const T*)h, (const T*)y_perm, slot_row, topk_gate,
-                                                     (const T*)y_shared, (T*)out, n, d, k);
+      launch_combine_t<moe::bf16, 1>(h, y_perm, slot_row, topk_gate, y_shared, out, n, d, k, shared_offsets, e, grid, s);
   } else {
     if (d % 4 == 0 && addr % 16 == 0)
-      moe::combine_kernel<float, 4><<<grid, 128, 0, s>>>((const float*)h, (const float*)y_perm, slot_row,
-                                                         topk_gate, (const float*)y_shared, (float*)out, n, d,
-                                                         k);
+      launch_combine_t<float, 4>(h, y_perm, slot_row, topk_gate, y_shared, out, n, d, k, shared_offsets, e, grid, s);
     else
-      moe::combine_kernel<float, 1><<<grid, 128, 0, s>>>((const float*)h, (const float*)y_perm, slot_row,
-                                                         topk_gate, (const float*)y_shared, (float*)out, n, d,
-                                                         k);
+      launch_combine_t<float, 1>(h, y_perm, slot_row, topk_gate, y_shared, out, n, d, k, shared_offsets, e, grid, s);
   }
   return launch_status();
 }

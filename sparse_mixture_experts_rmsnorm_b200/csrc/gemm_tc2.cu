@@ -97,7 +97,8 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                    const __grid_constant__ CUtensorMap map_b2, const TcArgs args) {
+                    const __grid_constant__ CUtensorMap map_b2, const __grid_constant__ CUtensorMap map_sb,
+                    const __grid_constant__ CUtensorMap map_sb2, const TcArgs args) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[P_STAGES];   // used in the even CTA
   __shared__ __align__(8) uint64_t empty_bar[P_STAGES];
@@ -151,16 +152,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     // ======================= TMA producer (both CTAs) =======================
     if (lane == 0) {
       tma_prefetch_map(&map_a);
-      tma_prefetch_map(rank == 1 && EPI == moe_host::EPI_SWIGLU ? &map_b2 : &map_b);
-      const CUtensorMap* bmap = (rank == 1 && EPI == moe_host::EPI_SWIGLU) ? &map_b2 : &map_b;
+      const bool second = rank == 1 && EPI == moe_host::EPI_SWIGLU;  // the up half of a SwiGLU tile
+      tma_prefetch_map(second ? &map_b2 : &map_b);
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
       bool ok = true;
       for (int t = first; t < total_tiles && ok; t += step) {
         const Tile tl = decode_tile<P_BM>(t, prefix_sh, offs_sh, G, args.out_cols);
+        const bool sh = tl.group == args.shared_group;  // the folded shared expert has its own weights
+        const CUtensorMap* bmap = sh ? (second ? &map_sb2 : &map_sb) : (second ? &map_b2 : &map_b);
         const int a_row = tl.row0 + (int)rank * 128;
-        const int b_row = tl.group * args.nout + tl.n0 + (EPI == moe_host::EPI_SWIGLU ? 0 : (int)rank * 128);
+        const int b_row = (sh ? 0 : tl.group * args.nout) + tl.n0 + (EPI == moe_host::EPI_SWIGLU ? 0 : (int)rank * 128);
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
                                  SITE_EMPTY)) {
@@ -303,7 +306,8 @@ static int resident_pairs() {
 
 template <int EPI>
 static moe_status launch_tc2_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
-                               const moe::TcArgs& args, int64_t pair_bound, cudaStream_t s) {
+                               const CUtensorMap& msb, const CUtensorMap& msb2, const moe::TcArgs& args,
+                               int64_t pair_bound, cudaStream_t s) {
   static bool attr_done[64] = {};
   int dev = current_device();
   if (dev < 64 && !attr_done[dev]) {
@@ -313,19 +317,21 @@ static moe_status launch_tc2_t(const CUtensorMap& ma, const CUtensorMap& mb, con
     attr_done[dev] = true;
   }
   const int64_t pairs = pair_bound < resident_pairs<EPI>() ? pair_bound : resident_pairs<EPI>();
-  moe::gemm_tc2_kernel<EPI><<<(unsigned)(2 * pairs), moe::P_THREADS, moe::P_SMEM_BYTES, s>>>(ma, mb, mb2, args);
+  moe::gemm_tc2_kernel<EPI><<<(unsigned)(2 * pairs), moe::P_THREADS, moe::P_SMEM_BYTES, s>>>(ma, mb, mb2, msb, msb2,
+                                                                                          args);
   return launch_status();
 }
 
 // Launch of the SM-pair kernel; maps and arguments come from launch_gemm_tc.
 moe_status launch_gemm_tc2(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
-                           const moe::TcArgs& args, int64_t max_rows, int groups_bound, cudaStream_t s) {
+                           const CUtensorMap& msb, const CUtensorMap& msb2, const moe::TcArgs& args, int64_t max_rows,
+                           int groups_bound, cudaStream_t s) {
   // upper bound on the pair tiles; the exact count lives on the device
   const int64_t m_pairs = (max_rows + moe::P_BM - 1) / moe::P_BM + groups_bound;
   const int64_t bound = m_pairs * args.n_tiles;
-  if (epi == EPI_SWIGLU) return launch_tc2_t<EPI_SWIGLU>(ma, mb, mb2, args, bound, s);
-  if (epi == EPI_STORE) return launch_tc2_t<EPI_STORE>(ma, mb, mb2, args, bound, s);
-  return launch_tc2_t<EPI_F32>(ma, mb, mb2, args, bound, s);
+  if (epi == EPI_SWIGLU) return launch_tc2_t<EPI_SWIGLU>(ma, mb, mb2, msb, msb2, args, bound, s);
+  if (epi == EPI_STORE) return launch_tc2_t<EPI_STORE>(ma, mb, mb2, msb, msb2, args, bound, s);
+  return launch_tc2_t<EPI_F32>(ma, mb, mb2, msb, msb2, args, bound, s);
 }
 
 }  // namespace moe_host

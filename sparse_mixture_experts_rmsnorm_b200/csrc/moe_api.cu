@@ -33,8 +33,9 @@ int sm_count() {
 // Workspace layout (every region 256-byte aligned)
 // ---------------------------------------------------------------------------
 struct Layout {
-  size_t hdr, xn, logits, idx, gate, counts, offsets, slot_row, row_token, hist, x_perm, act, y_perm, y_shared,
-      total;
+  size_t hdr, xn, logits, idx, gate, counts, offsets, offsets_ext, slot_row, row_token, hist, x_perm, act, y_perm,
+      y_shared, total;
+  bool fold;         // the shared expert runs as one more group of the routed GEMMs
   int64_t rows;      // R: rows of the expert-sorted buffers
   int64_t act_elems; // max(R * H, N * Hs)
 };
@@ -52,7 +53,12 @@ static Layout layout_of(const moe_config* c) {
   int64_t R = N * k;
   if (cap >= 0 && E * cap < R) R = E * cap;
   L.rows = R;
-  L.act_elems = R * c->d_ff;
+  // bf16 layers with a shared expert as wide as the routed ones fold it into
+  // the routed GEMMs: its N rows follow the R routed rows in x_perm, act and y_perm
+  L.fold = c->dtype == MOE_BF16 && c->d_ff_shared > 0 && c->d_ff_shared == c->d_ff &&
+           c->n_experts < moe::TC_MAX_GROUPS;
+  const int64_t Rx = R + (L.fold ? N : 0);
+  L.act_elems = Rx * c->d_ff;
   if (N * (int64_t)c->d_ff_shared > L.act_elems) L.act_elems = N * c->d_ff_shared;
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -67,13 +73,14 @@ static Layout layout_of(const moe_config* c) {
   L.gate = take(N * k * 4);
   L.counts = take(E * 4);
   L.offsets = take((E + 1) * 4);
+  L.offsets_ext = take((E + 2) * 4);
   L.slot_row = take(N * k * 4);
   L.row_token = take(N * k * 4);
   L.hist = take(permute_hist_ints(N * k, (int)E) * 4);
-  L.x_perm = take(R * d * es);
+  L.x_perm = take(Rx * d * es);
   L.act = take(L.act_elems * es);
-  L.y_perm = take(R * d * es);
-  L.y_shared = take(c->d_ff_shared > 0 ? N * d * es : 0);
+  L.y_perm = take(Rx * d * es);
+  L.y_shared = take(c->d_ff_shared > 0 && !L.fold ? N * d * es : 0);
   L.total = o;
   return L;
 }
@@ -286,12 +293,36 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const 
   MOE_TRY(mark(trace ? trace->start : nullptr));
   MOE_TRY(route_impl(cfg, h, w->norm_w, w->w_router, bias, xn, scores, idx, gate, counts, ws, s));
   MOE_TRY(mark(trace ? trace->routed : nullptr));
+  const int R = (int)L.rows;
+  const int N = cfg->n_tokens;
+  void* act = wsp(ws, L.act);
+  int32_t* hdr = (int32_t*)wsp(ws, L.hdr);
+  if (L.fold) {
+    // routed experts 0..E-1 plus the shared expert as group E over all N tokens
+    int32_t* offs_ext = (int32_t*)wsp(ws, L.offsets_ext);
+    MOE_TRY(launch_permute(idx, N, cfg->top_k, cfg->n_experts, (int)capacity_of(cfg), (int32_t*)wsp(ws, L.hist),
+                           offsets, slot_row, row_token, s, offs_ext, N));
+    MOE_TRY(launch_gather(cfg->dtype, xn, row_token, offsets, cfg->n_experts, x_perm, R, cfg->d_model, s, N));
+    MOE_TRY(mark(trace ? trace->permuted : nullptr));
+    if (N > 0) {
+      MOE_TRY(launch_gemm_tc(EPI_SWIGLU, x_perm, w->w_gate, w->w_up, offs_ext, cfg->n_experts + 1, R + N, cfg->d_ff,
+                             cfg->d_model, act, cfg->d_ff, hdr, s, w->ws_gate, w->ws_up));
+      MOE_TRY(mark(trace ? trace->gate_up : nullptr));
+      MOE_TRY(launch_gemm_tc(EPI_STORE, act, w->w_down, nullptr, offs_ext, cfg->n_experts + 1, R + N, cfg->d_model,
+                             cfg->d_ff, y_perm, cfg->d_model, hdr, s, w->ws_down, nullptr));
+    } else {
+      MOE_TRY(mark(trace ? trace->gate_up : nullptr));
+    }
+    MOE_TRY(mark(trace ? trace->down : nullptr));
+    MOE_TRY(mark(trace ? trace->shared : nullptr));  // included in the two launches above
+    MOE_TRY(launch_combine(cfg->dtype, h, y_perm, slot_row, gate, nullptr, out, N, cfg->d_model, cfg->top_k, s,
+                           offs_ext, cfg->n_experts));
+    MOE_TRY(mark(trace ? trace->combined : nullptr));
+    return MOE_OK;
+  }
   MOE_TRY(permute_impl(cfg, idx, xn, offsets, slot_row, row_token, x_perm, ws, s));
   MOE_TRY(mark(trace ? trace->permuted : nullptr));
-  const int R = (int)L.rows;
   if (R > 0) {
-    void* act = wsp(ws, L.act);
-    int32_t* hdr = (int32_t*)wsp(ws, L.hdr);
     if (use_tc(cfg)) {
       MOE_TRY(launch_gemm_tc(EPI_SWIGLU, x_perm, w->w_gate, w->w_up, offsets, cfg->n_experts, R, cfg->d_ff,
                              cfg->d_model, act, cfg->d_ff, hdr, s));
@@ -309,12 +340,10 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const 
     MOE_TRY(mark(trace ? trace->gate_up : nullptr));
   }
   MOE_TRY(mark(trace ? trace->down : nullptr));
-  if (shared && cfg->n_tokens > 0)
-    MOE_TRY(ffn_impl(cfg, 1, nullptr, cfg->n_tokens, xn, w->ws_gate, w->ws_up, w->ws_down, cfg->d_ff_shared,
-                     y_shared, ws, s));
+  if (shared && N > 0)
+    MOE_TRY(ffn_impl(cfg, 1, nullptr, N, xn, w->ws_gate, w->ws_up, w->ws_down, cfg->d_ff_shared, y_shared, ws, s));
   MOE_TRY(mark(trace ? trace->shared : nullptr));
-  MOE_TRY(launch_combine(cfg->dtype, h, y_perm, slot_row, gate, y_shared, out, cfg->n_tokens, cfg->d_model,
-                         cfg->top_k, s));
+  MOE_TRY(launch_combine(cfg->dtype, h, y_perm, slot_row, gate, y_shared, out, N, cfg->d_model, cfg->top_k, s));
   MOE_TRY(mark(trace ? trace->combined : nullptr));
   return MOE_OK;
 }

@@ -33,18 +33,24 @@ moe_status launch_hash_route(const int64_t* token_ids, int32_t* topk_idx, float*
 
 // a4: stable counting sort of the N*k slots by expert with optional capacity.
 //   hist: workspace of permute_hist_ints(n*k, e) int32.
+//   offsets_ext != nullptr: also writes offsets_ext[0..E] = offsets and
+//   offsets_ext[E+1] = offsets[E] + extra (a trailing group of `extra` rows).
 size_t permute_hist_ints(int64_t slots, int e);
 moe_status launch_permute(const int32_t* topk_idx, int n, int k, int e, int cap, int32_t* hist,
-                          int32_t* offsets, int32_t* slot_row, int32_t* row_token, cudaStream_t s);
+                          int32_t* offsets, int32_t* slot_row, int32_t* row_token, cudaStream_t s,
+                          int32_t* offsets_ext = nullptr, int extra = 0);
 
-// a5: x_perm[r] = xn[row_token[r]] for r < offsets[e] (device count).
+// a5: x_perm[r] = xn[row_token[r]] for r < R = offsets[e] (device count),
+// and x_perm[R + t] = xn[t] for t < shared_rows (the folded shared expert).
 moe_status launch_gather(int dtype, const void* xn, const int32_t* row_token, const int32_t* offsets, int e,
-                         void* x_perm, int max_rows, int d, cudaStream_t s);
+                         void* x_perm, int max_rows, int d, cudaStream_t s, int shared_rows = 0);
 
-// a9: out = h + sum_j gate_j * y_perm[slot_row] (+ y_shared).
+// a9: out = h + sum_j gate_j * y_perm[slot_row] (+ y_shared).  With
+// shared_offsets != nullptr the shared rows are y_perm rows from
+// shared_offsets[e] on (the folded shared expert) and y_shared is ignored.
 moe_status launch_combine(int dtype, const void* h, const void* y_perm, const int32_t* slot_row,
                           const float* topk_gate, const void* y_shared, void* out, int n, int d, int k,
-                          cudaStream_t s);
+                          cudaStream_t s, const int32_t* shared_offsets = nullptr, int e = 0);
 
 // a10: bias[e] += gamma * sign(target - counts[e]).
 moe_status launch_bias_update(int e, const int32_t* counts, float target, float gamma, float* bias,
@@ -65,9 +71,11 @@ moe_status launch_gemm_simt(int dtype, int epi, const void* a, const void* b, co
 // The same grouped GEMM on the tcgen05 tensor cores (bf16 operands only,
 // TMA-fed, TMEM accumulators, persistent over the SMs).  k % 8 == 0.
 //   hdr: workspace header that receives a device time-out, if any.
+//   sb, sb2 != nullptr: the last group is the shared expert, with its own
+//   [nout][k] weights sb (gate or down) and sb2 (up).
 moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2, const int32_t* offsets,
-                          int groups, int max_rows, int nout, int k, void* c, int ldc, int32_t* hdr,
-                          cudaStream_t s);
+                          int groups, int max_rows, int nout, int k, void* c, int ldc, int32_t* hdr, cudaStream_t s,
+                          const void* sb = nullptr, const void* sb2 = nullptr);
 
 // A block that waits, with the bounded wait of the pipelined kernels, on a
 // barrier that nothing completes.

@@ -72,7 +72,8 @@ __global__ void __launch_bounds__(kPermWarps * 32) chunk_hist_kernel(const int32
 //      expert e; the row total is count_e.
 //   2. kept_e = min(count_e, cap); offsets = exclusive scan of kept (E+1).
 __global__ void __launch_bounds__(1024) hist_scan_kernel(int32_t* __restrict__ hist, int E, int nchunks, int cap,
-                                                         int32_t* __restrict__ offsets) {
+                                                         int32_t* __restrict__ offsets,
+                                                         int32_t* __restrict__ offsets_ext, int extra) {
   __shared__ int32_t kept_sh[1024];
   __shared__ int32_t warp_sum[32];
   const int lane = lane_id(), warp = warp_id();
@@ -117,6 +118,13 @@ __global__ void __launch_bounds__(1024) hist_scan_kernel(int32_t* __restrict__ h
   const int32_t excl = x - k + (warp > 0 ? warp_sum[warp - 1] : 0);
   if (tid < E) offsets[tid] = excl;
   if (tid == E - 1) offsets[E] = excl + k;
+  if (offsets_ext != nullptr) {  // the same offsets plus a trailing group of `extra` rows
+    if (tid < E) offsets_ext[tid] = excl;
+    if (tid == E - 1) {
+      offsets_ext[E] = excl + k;
+      offsets_ext[E + 1] = excl + k + extra;
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kPermWarps * 32) chunk_scatter_kernel(
@@ -141,17 +149,20 @@ __global__ void __launch_bounds__(kPermWarps * 32) chunk_scatter_kernel(
   });
 }
 
-// a5: x_perm[r] = xn[row_token[r]] for r < offsets[E].  One block per row,
+// a5: x_perm[r] = xn[row_token[r]] for r < R = offsets[E], then
+// x_perm[R + t] = xn[t] for t < shared_rows.  One block per row,
 // grid-stride; VEC elements per 16-byte access when the row allows it.
 template <typename V>
 __global__ void __launch_bounds__(128) gather_rows_kernel(const V* __restrict__ xn,
                                                           const int32_t* __restrict__ row_token,
                                                           const int32_t* __restrict__ offsets, int E,
-                                                          V* __restrict__ x_perm, int row_vecs) {
-  const int rows = offsets[E];
+                                                          V* __restrict__ x_perm, int row_vecs, int shared_rows) {
+  const int routed = offsets[E];
+  const int rows = routed + shared_rows;
   for (int r = blockIdx.x; r < rows; r += gridDim.x) {
-    const V* src = xn + (size_t)row_token[r] * row_vecs;
+    const V* src = xn + (size_t)(r < routed ? row_token[r] : r - routed) * row_vecs;
     V* dst = x_perm + (size_t)r * row_vecs;
+#pragma unroll 4
     for (int i = threadIdx.x; i < row_vecs; i += blockDim.x) dst[i] = src[i];
   }
 }
@@ -165,37 +176,42 @@ static inline int64_t n_chunks(int64_t slots) { return (slots + moe::kChunk - 1)
 size_t permute_hist_ints(int64_t slots, int e) { return (size_t)(n_chunks(slots) > 0 ? n_chunks(slots) : 1) * e; }
 
 moe_status launch_permute(const int32_t* topk_idx, int n, int k, int e, int cap, int32_t* hist,
-                          int32_t* offsets, int32_t* slot_row, int32_t* row_token, cudaStream_t s) {
+                          int32_t* offsets, int32_t* slot_row, int32_t* row_token, cudaStream_t s,
+                          int32_t* offsets_ext, int extra) {
   const int64_t slots = (int64_t)n * k;
   const int64_t nch = n_chunks(slots);
   if (nch == 0) {
     if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (e + 1), s) != cudaSuccess) return MOE_ERR_CUDA;
+    // no slots means no tokens, so the trailing group is empty too (extra == 0)
+    if (offsets_ext != nullptr && cudaMemsetAsync(offsets_ext, 0, sizeof(int32_t) * (e + 2), s) != cudaSuccess)
+      return MOE_ERR_CUDA;
     return MOE_OK;
   }
   const int blocks = (int)((nch + moe::kPermWarps - 1) / moe::kPermWarps);
   const size_t smem = sizeof(int32_t) * e * moe::kPermWarps;
   moe::chunk_hist_kernel<<<blocks, moe::kPermWarps * 32, smem, s>>>(topk_idx, slots, e, (int)nch, hist);
-  moe::hist_scan_kernel<<<1, 1024, 0, s>>>(hist, e, (int)nch, cap, offsets);
+  moe::hist_scan_kernel<<<1, 1024, 0, s>>>(hist, e, (int)nch, cap, offsets, offsets_ext, extra);
   moe::chunk_scatter_kernel<<<blocks, moe::kPermWarps * 32, smem, s>>>(topk_idx, slots, k, e, (int)nch, cap,
                                                                        hist, offsets, slot_row, row_token);
   return launch_status();
 }
 
 moe_status launch_gather(int dtype, const void* xn, const int32_t* row_token, const int32_t* offsets, int e,
-                         void* x_perm, int max_rows, int d, cudaStream_t s) {
+                         void* x_perm, int max_rows, int d, cudaStream_t s, int shared_rows) {
+  max_rows += shared_rows;
   if (max_rows == 0) return MOE_OK;
   const size_t row_bytes = (size_t)d * (dtype == MOE_BF16 ? 2 : 4);
   int grid = max_rows < sm_count() * 16 ? max_rows : sm_count() * 16;
   const uintptr_t addr = (uintptr_t)xn | (uintptr_t)x_perm;
   if (row_bytes % 16 == 0 && addr % 16 == 0)
     moe::gather_rows_kernel<uint4><<<grid, 128, 0, s>>>((const uint4*)xn, row_token, offsets, e, (uint4*)x_perm,
-                                                        (int)(row_bytes / 16));
+                                                        (int)(row_bytes / 16), shared_rows);
   else if (row_bytes % 4 == 0 && addr % 4 == 0)
     moe::gather_rows_kernel<uint32_t><<<grid, 128, 0, s>>>((const uint32_t*)xn, row_token, offsets, e,
-                                                           (uint32_t*)x_perm, (int)(row_bytes / 4));
+                                                           (uint32_t*)x_perm, (int)(row_bytes / 4), shared_rows);
   else
     moe::gather_rows_kernel<uint16_t><<<grid, 128, 0, s>>>((const uint16_t*)xn, row_token, offsets, e,
-                                                           (uint16_t*)x_perm, (int)(row_bytes / 2));
+                                                           (uint16_t*)x_perm, (int)(row_bytes / 2), shared_rows);
   return launch_status();
 }
 

@@ -298,6 +298,9 @@ def test_device_wait_times_out_and_reports(torch_cuda):
          skew=(5, 8.0, 2.0)),
     dict(n_tokens=97, d_model=128, n_experts=64, top_k=6, d_ff=64, d_ff_shared=64,
          bias=("uniform", -0.01, 0.01)),
+    # shared expert as wide as the routed ones (it runs inside the routed GEMMs) plus drops
+    dict(n_tokens=400, d_model=256, n_experts=8, top_k=2, d_ff=128, d_ff_shared=128, capacity_factor=0.8,
+         skew=(2, 8.0, 2.5)),
 ])
 def test_small_bf16_layer_every_output(torch_cuda, over):
     cfg = mi.LayerConfig(name="small", dtype="bf16", seed=4, **over)
