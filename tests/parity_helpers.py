@@ -114,7 +114,7 @@ def check_routing(gpu: dict, ref: dict, k: int, gate_tol: float = 1e-5):
     assert np.array_equal(gs[same_set], rs[same_set])
     np.testing.assert_allclose(gpu["topk_gate"][ok], ref["gates"][ok], rtol=0, atol=gate_tol)
     assert np.all(gpu["topk_gate"] >= 0)
-    np.testing.assert_allclose(gpu["topk_gate"].sum(1), 1.0, atol=2e-6)
+    np.testing.assert_allclose(gpu["topk_gate"].astype(np.float64).sum(1), 1.0, atol=2e-6)
     E = ref["scores"].shape[1]
     counts = np.bincount(gi.ravel(), minlength=E)
     assert np.array_equal(gpu["counts"].astype(np.int64), counts)

@@ -15,7 +15,7 @@ import pytest
 import moe_inputs as mi
 import oracle
 from parity_helpers import (BF16_REL_RMS, F32_MAX_ABS, bf16_rel_rms_err, check_permutation, check_routing,
-                            lib_config, oracle_routing, rel_rms_err, run_gpu_layer, to_np)
+                            lib_config, oracle_routing, rel_rms_err, run_gpu_layer, tie_masks, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -347,3 +347,22 @@ def test_layer_forward_replays_from_a_cuda_graph(torch_cuda, name):
         assert torch.equal(out, eager)
     st, info = moe.moe_check_device_error(ws)
     assert st == 0, info
+
+
+# ----------------------------------------------------------------- the largest routing the ABI allows
+
+@pytest.mark.parametrize("n_tokens", [300, 700])  # router on the CUDA cores, then on the tensor cores
+def test_route_with_1024_experts_and_top_32(torch_cuda, n_tokens):
+    # with 1024 experts neighbouring keys often fall within 1e-6 of each other:
+    # those tokens are compared as sets only (check_routing), and such ties are
+    # counted here
+    cfg = mi.LayerConfig(name="wide", n_tokens=n_tokens, d_model=256, n_experts=1024, top_k=32, d_ff=64,
+                         bias=("uniform", -1e-4, 1e-4), router_sigma=0.1, seed=8)
+    g = run_gpu_layer(cfg)
+    ref = oracle_routing(cfg)
+    np.testing.assert_array_equal(g["xn"], ref["xn"])
+    np.testing.assert_allclose(g["scores"], ref["scores"], rtol=2e-5, atol=1e-10)
+    set_amb, _ = tie_masks(ref["key"], cfg.top_k)
+    skipped = check_routing(g, ref, cfg.top_k)
+    assert set_amb.mean() < 0.05 and skipped < 0.25 * n_tokens, (set_amb.mean(), skipped)
+    check_permutation(g, cfg.n_experts, -1)
