@@ -21,7 +21,9 @@
 //               32 TMEM lanes = rows its rank allows), SwiGLU or plain
 //               conversion, masked stores of the rows inside the group.
 // The two accumulators let the epilogue of one tile overlap the main loop
-// of the next.  For SwiGLU, B holds 128 gate rows then 128 up rows of the
+// of the next.  A tile of at most 64 rows (a ragged expert's last tile, or
+// every tile of a decode step) runs as M = 64 MMAs; its accumulator keeps row
+// r in TMEM lane (r / 16) * 32 + r % 16, the first 16 lanes of each quarter.  For SwiGLU, B holds 128 gate rows then 128 up rows of the
 // same hidden units, so one N = 256 MMA produces both halves.
 // Tiles are numbered group-major, then n-tile, then m-tile, so CTAs working
 // at the same time share weight tiles through L2.
@@ -156,6 +158,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t bphase = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        const Tile tl = decode_tile<TC_BM>(t, prefix_sh, offs_sh, G, args.out_cols);
+        // a tile of at most 64 rows runs as M = 64 MMAs (half the rows of work)
+        const uint32_t id = (tl.row_end - tl.row0 <= 64) ? tc_idesc(64, TC_BN) : idesc;
         if (!mbar_wait_bounded(&tempty_bar[buf], bphase ^ 1u, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
                                SITE_TMEM_EMPTY))
           break;
@@ -173,7 +178,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           const uint64_t bdesc = sw128_desc(sa + TC_A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < TC_BK / 16; ++kk)  // K = 16 per MMA: 32 bytes further along the row
-            tc_mma(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc, (kb | kk) != 0);
+            tc_mma(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), id, (kb | kk) != 0);
           tc_commit(&empty_bar[stage]);
           if (++stage == TC_STAGES) {
             stage = 0;
@@ -207,8 +212,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * TC_BN);
-      const int row = tl.row0 + r_local;
-      epilogue_row<EPI>(args, tbase, row, row < tl.row_end, tl.n0);
+      // M = 64 accumulators keep row r in lane (r / 16) * 32 + r % 16: lanes
+      // 0..15 of each warp's quarter
+      const bool half = tl.row_end - tl.row0 <= 64;
+      const int row = half ? tl.row0 + quarter * 16 + (lane & 15) : tl.row0 + r_local;
+      epilogue_row<EPI>(args, tbase, row, row < tl.row_end && (!half || lane < 16), tl.n0);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty_bar[buf]);
