@@ -54,14 +54,22 @@ def test_workspace_size_grows_with_shape_and_rejects_bad_configs():
 
 
 def test_workspace_bytes_match_the_documented_regions():
-    c = _cfg(dtype="bf16", n_tokens=1000, d_model=512, n_experts=16, top_k=4, d_ff=384, d_ff_shared=256)
+    N, d, E, k, H, Hs = 1000, 512, 16, 4, 384, 256
+    routing = N * E * 4 + 4 * N * k * 4  # logits, idx, gate, slot_row, row_token
+    # bf16: xn, routing, x_perm, act, y_perm, y_shared
+    c = _cfg(dtype="bf16", n_tokens=N, d_model=d, n_experts=E, top_k=k, d_ff=H, d_ff_shared=Hs)
     R = c.rows
-    es = 2
-    need = (c.n_tokens * c.d_model * es + c.n_tokens * c.n_experts * 4 + 4 * c.n_tokens * c.top_k * 4
-            + R * c.d_model * es * 2 + max(R * c.d_ff, c.n_tokens * c.d_ff_shared) * es
-            + c.n_tokens * c.d_model * es)
-    got = moe.workspace_size(c)
-    assert need <= got <= need + 64 * 1024
+    need = N * d * 2 + routing + 2 * R * d * 2 + max(R * H, N * Hs) * 2 + N * d * 2
+    assert need <= moe.workspace_size(c) <= need + 64 * 1024
+    # fp32: the same regions in 4-byte elements
+    f = _cfg(dtype="f32", n_tokens=N, d_model=d, n_experts=E, top_k=k, d_ff=H, d_ff_shared=Hs)
+    need32 = N * d * 4 + routing + 2 * R * d * 4 + max(R * H, N * Hs) * 4 + N * d * 4
+    assert need32 <= moe.workspace_size(f) <= need32 + 64 * 1024
+    # bf16 with a shared expert as wide as the routed ones: it is one more
+    # group of N rows in x_perm, act and y_perm, and there is no separate y_shared
+    g = _cfg(dtype="bf16", n_tokens=N, d_model=d, n_experts=E, top_k=k, d_ff=H, d_ff_shared=H)
+    need_f = N * d * 2 + routing + 2 * (R + N) * d * 2 + (R + N) * H * 2
+    assert need_f <= moe.workspace_size(g) <= need_f + 64 * 1024
 
 
 def test_host_validation_before_any_launch():
