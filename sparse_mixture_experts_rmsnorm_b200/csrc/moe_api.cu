@@ -2,7 +2,6 @@
 // layout and the order of the kernels on the caller's stream.  No entry
 // point allocates device memory, and only moe_check_device_error
 // synchronises.
-#include <stdio.h>
 
 #include "moe_common.cuh"
 #include "moe_kernels.h"

@@ -97,6 +97,19 @@ def test_tiny_fp32_staged_calls_equal_layer_forward(torch_cuda):
     np.testing.assert_array_equal(to_np(x_perm), to_np(xn)[g["row_token"]])
 
 
+def test_tiny_fp32_layer_with_shared_expert_and_capacity(torch_cuda):
+    # the CUDA-core path with an always-on shared expert and dropped slots
+    cfg = mi.CONFIGS["tiny_fp32"].with_(d_ff_shared=96, capacity_factor=0.75, skew=(4, 8.0, 3.0), seed=3)
+    g = run_gpu_layer(cfg)
+    ref = _full_oracle(cfg)
+    check_routing(g, {"key": ref["key"], "idx": ref["idx"], "gates": ref["gates"], "scores": ref["scores"]},
+                  cfg.top_k)
+    check_permutation(g, cfg.n_experts, cfg.capacity)
+    assert (g["slot_row"] < 0).any()
+    err = np.max(np.abs(g["out"] - ref["out64"]))
+    assert err <= F32_MAX_ABS, err
+
+
 def test_single_expert_and_dense_identities(torch_cuda):
     # E = 1, k = 1: the textbook SwiGLU FFN; k = E (zero bias): dense softmax-weighted sum.
     for over in (dict(n_experts=1, top_k=1), dict(n_experts=4, top_k=4), dict(n_experts=8, top_k=8)):
