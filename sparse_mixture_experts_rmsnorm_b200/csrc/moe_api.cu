@@ -129,6 +129,8 @@ static bool router_on_tc(const moe_config* c) {
   return use_tc(c) && c->n_experts >= 64 && c->n_tokens >= 512;
 }
 
+// counts == nullptr: no counts here (the layer forward takes them from the
+// permute's scan instead, which needs no atomics).
 static moe_status route_impl(const moe_config* c, const void* h, const void* norm_w, const void* w_router,
                              const float* bias, void* xn, float* scores, int32_t* topk_idx, float* topk_gate,
                              int32_t* counts, void* ws, cudaStream_t s) {
@@ -150,11 +152,12 @@ static moe_status route_impl(const moe_config* c, const void* h, const void* nor
 }
 
 static moe_status permute_impl(const moe_config* c, const int32_t* topk_idx, const void* xn, int32_t* offsets,
-                               int32_t* slot_row, int32_t* row_token, void* x_perm, void* ws, cudaStream_t s) {
+                               int32_t* slot_row, int32_t* row_token, void* x_perm, void* ws, cudaStream_t s,
+                               int32_t* counts = nullptr) {
   const Layout L = layout_of(c);
   const int cap = (int)capacity_of(c);
   MOE_TRY(launch_permute(topk_idx, c->n_tokens, c->top_k, c->n_experts, cap, (int32_t*)wsp(ws, L.hist), offsets,
-                         slot_row, row_token, s));
+                         slot_row, row_token, s, nullptr, 0, counts));
   return launch_gather(c->dtype, xn, row_token, offsets, c->n_experts, x_perm, (int)L.rows, c->d_model, s);
 }
 
@@ -290,7 +293,8 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const 
     return MOE_OK;
   };
   MOE_TRY(mark(trace ? trace->start : nullptr));
-  MOE_TRY(route_impl(cfg, h, w->norm_w, w->w_router, bias, xn, scores, idx, gate, counts, ws, s));
+  // the counts come from the permute's scan below
+  MOE_TRY(route_impl(cfg, h, w->norm_w, w->w_router, bias, xn, scores, idx, gate, nullptr, ws, s));
   MOE_TRY(mark(trace ? trace->routed : nullptr));
   const int R = (int)L.rows;
   const int N = cfg->n_tokens;
@@ -300,7 +304,7 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const 
     // routed experts 0..E-1 plus the shared expert as group E over all N tokens
     int32_t* offs_ext = (int32_t*)wsp(ws, L.offsets_ext);
     MOE_TRY(launch_permute(idx, N, cfg->top_k, cfg->n_experts, (int)capacity_of(cfg), (int32_t*)wsp(ws, L.hist),
-                           offsets, slot_row, row_token, s, offs_ext, N));
+                           offsets, slot_row, row_token, s, offs_ext, N, counts));
     MOE_TRY(launch_gather(cfg->dtype, xn, row_token, offsets, cfg->n_experts, x_perm, R, cfg->d_model, s, N));
     MOE_TRY(mark(trace ? trace->permuted : nullptr));
     if (N > 0) {
@@ -319,7 +323,7 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const 
     MOE_TRY(mark(trace ? trace->combined : nullptr));
     return MOE_OK;
   }
-  MOE_TRY(permute_impl(cfg, idx, xn, offsets, slot_row, row_token, x_perm, ws, s));
+  MOE_TRY(permute_impl(cfg, idx, xn, offsets, slot_row, row_token, x_perm, ws, s, counts));
   MOE_TRY(mark(trace ? trace->permuted : nullptr));
   if (R > 0) {
     if (use_tc(cfg)) {

@@ -22,7 +22,8 @@ moe_status launch_rmsnorm_router(int dtype, const void* h, const void* norm_w, c
                                  float* logits, int n, int d, int e, float eps, cudaStream_t s);
 
 // a3: softmax over the router logits, top-k on score + bias, renormalised
-// gates and the per-expert counts (counts are zeroed here first).
+// gates and the per-expert counts (counts are zeroed here first; with
+// counts == nullptr none are taken).
 moe_status launch_topk(const float* logits, const float* bias, float* scores, int32_t* topk_idx,
                        float* topk_gate, int32_t* counts, int n, int e, int k, cudaStream_t s);
 
@@ -35,10 +36,12 @@ moe_status launch_hash_route(const int64_t* token_ids, int32_t* topk_idx, float*
 //   hist: workspace of permute_hist_ints(n*k, e) int32.
 //   offsets_ext != nullptr: also writes offsets_ext[0..E] = offsets and
 //   offsets_ext[E+1] = offsets[E] + extra (a trailing group of `extra` rows).
+//   counts != nullptr: also writes the per-expert slot counts (before the
+//   capacity cut), the `counts` that launch_topk would give.
 size_t permute_hist_ints(int64_t slots, int e);
 moe_status launch_permute(const int32_t* topk_idx, int n, int k, int e, int cap, int32_t* hist,
                           int32_t* offsets, int32_t* slot_row, int32_t* row_token, cudaStream_t s,
-                          int32_t* offsets_ext = nullptr, int extra = 0);
+                          int32_t* offsets_ext = nullptr, int extra = 0, int32_t* counts = nullptr);
 
 // a5: x_perm[r] = xn[row_token[r]] for r < R = offsets[e] (device count),
 // and x_perm[R + t] = xn[t] for t < shared_rows (the folded shared expert).

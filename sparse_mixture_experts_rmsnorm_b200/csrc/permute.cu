@@ -69,30 +69,52 @@ __global__ void __launch_bounds__(kPermWarps * 32) chunk_hist_kernel(const int32
 // One block of 1024 threads.
 //   1. Each warp takes whole experts: the exclusive scan of hist[e][*] over
 //      the chunks, in place, gives every chunk the rank of its first slot of
-//      expert e; the row total is count_e.
+//      expert e; the row total is count_e (also written to `counts` when
+//      given).  The warp loads 32 * kScanPer chunk counts with coalesced,
+//      independent loads, scans them as kScanPer warp scans in registers and
+//      stores them back coalesced: one memory round trip per 32 * kScanPer
+//      chunks.
 //   2. kept_e = min(count_e, cap); offsets = exclusive scan of kept (E+1).
+constexpr int kScanPer = 8;
+
 __global__ void __launch_bounds__(1024) hist_scan_kernel(int32_t* __restrict__ hist, int E, int nchunks, int cap,
                                                          int32_t* __restrict__ offsets,
-                                                         int32_t* __restrict__ offsets_ext, int extra) {
+                                                         int32_t* __restrict__ offsets_ext, int extra,
+                                                         int32_t* __restrict__ counts) {
   __shared__ int32_t kept_sh[1024];
   __shared__ int32_t warp_sum[32];
   const int lane = lane_id(), warp = warp_id();
   for (int e = warp; e < E; e += 32) {
     int32_t* row = hist + (int64_t)e * nchunks;
     int32_t carry = 0;
-    for (int c0 = 0; c0 < nchunks; c0 += 32) {
-      const int c = c0 + lane;
-      const int32_t v = (c < nchunks) ? row[c] : 0;
-      int32_t x = v;
+    for (int c0 = 0; c0 < nchunks; c0 += 32 * kScanPer) {
+      int32_t v[kScanPer];
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        int32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
+      for (int i = 0; i < kScanPer; ++i) {
+        const int c = c0 + 32 * i + lane;
+        v[i] = (c < nchunks) ? row[c] : 0;
       }
-      if (c < nchunks) row[c] = carry + x - v;
-      carry += __shfl_sync(0xffffffffu, x, 31);
+#pragma unroll
+      for (int i = 0; i < kScanPer; ++i) {
+        int32_t x = v[i];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        v[i] = carry + x - v[i];
+        carry += __shfl_sync(0xffffffffu, x, 31);
+      }
+#pragma unroll
+      for (int i = 0; i < kScanPer; ++i) {
+        const int c = c0 + 32 * i + lane;
+        if (c < nchunks) row[c] = v[i];
+      }
     }
-    if (lane == 0) kept_sh[e] = (cap >= 0 && carry > cap) ? cap : carry;
+    if (lane == 0) {
+      kept_sh[e] = (cap >= 0 && carry > cap) ? cap : carry;
+      if (counts != nullptr) counts[e] = carry;
+    }
   }
   __syncthreads();
   const int tid = threadIdx.x;
@@ -177,7 +199,7 @@ size_t permute_hist_ints(int64_t slots, int e) { return (size_t)(n_chunks(slots)
 
 moe_status launch_permute(const int32_t* topk_idx, int n, int k, int e, int cap, int32_t* hist,
                           int32_t* offsets, int32_t* slot_row, int32_t* row_token, cudaStream_t s,
-                          int32_t* offsets_ext, int extra) {
+                          int32_t* offsets_ext, int extra, int32_t* counts) {
   const int64_t slots = (int64_t)n * k;
   const int64_t nch = n_chunks(slots);
   if (nch == 0) {
@@ -185,12 +207,13 @@ moe_status launch_permute(const int32_t* topk_idx, int n, int k, int e, int cap,
     // no slots means no tokens, so the trailing group is empty too (extra == 0)
     if (offsets_ext != nullptr && cudaMemsetAsync(offsets_ext, 0, sizeof(int32_t) * (e + 2), s) != cudaSuccess)
       return MOE_ERR_CUDA;
+    if (counts != nullptr && cudaMemsetAsync(counts, 0, sizeof(int32_t) * e, s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
   }
   const int blocks = (int)((nch + moe::kPermWarps - 1) / moe::kPermWarps);
   const size_t smem = sizeof(int32_t) * e * moe::kPermWarps;
   moe::chunk_hist_kernel<<<blocks, moe::kPermWarps * 32, smem, s>>>(topk_idx, slots, e, (int)nch, hist);
-  moe::hist_scan_kernel<<<1, 1024, 0, s>>>(hist, e, (int)nch, cap, offsets, offsets_ext, extra);
+  moe::hist_scan_kernel<<<1, 1024, 0, s>>>(hist, e, (int)nch, cap, offsets, offsets_ext, extra, counts);
   moe::chunk_scatter_kernel<<<blocks, moe::kPermWarps * 32, smem, s>>>(topk_idx, slots, k, e, (int)nch, cap,
                                                                        hist, offsets, slot_row, row_token);
   return launch_status();

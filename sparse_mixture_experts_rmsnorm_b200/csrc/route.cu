@@ -22,7 +22,8 @@ namespace moe {
 // r = fl32(1 / sqrt(ms + eps)) is taken in fp64 and rounded once, then
 // xn = round(fl32(fl32(h * r) * w)), so the storage rounding is decided in fp32.
 //
-// One block per token (grid-stride), V elements per 16-byte access.  The
+// One block per token (grid-stride), V elements per 16-byte access; the row
+// comes in with cp.async, all of its copies in flight at once.  The
 // row is staged in shared memory in its own dtype; when `logits` is given, the
 // block's warps then take the router dot products of the rounded xn row
 // with experts [e0, e0 + epb) (e0 = blockIdx.y * epb), one expert per warp
@@ -67,16 +68,32 @@ __global__ void __launch_bounds__(256) rmsnorm_router_kernel(const T* __restrict
   const int e0 = blockIdx.y * epb;
   const int e1 = min(E, e0 + epb);
   const int warps = blockDim.x >> 5;
+  const int step = blockDim.x * V;  // elements per pass of the block
   for (int t = blockIdx.x; t < n; t += gridDim.x) {
     const T* hr = h + (size_t)t * d;
     double acc = 0.0;
-    for (int i = threadIdx.x * V; i < d; i += blockDim.x * V) {
-      const Vec<T, V> x = ld_vec<T, V>(hr + i);
-      float f[V];
-      vec_to_f32(x, f);
+    if (V * sizeof(T) == 16) {
+      // every 16-byte copy of the row in flight at once (cp.async, no
+      // registers held); each thread then reads back the elements it copied,
+      // in increasing order
+      for (int i = threadIdx.x * V; i < d; i += step)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(row + i)), "l"(hr + i) : "memory");
+      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+      for (int i = threadIdx.x * V; i < d; i += step) {
+        float f[V];
+        vec_to_f32(ld_vec<T, V>(row + i), f);
 #pragma unroll
-      for (int j = 0; j < V; ++j) acc += (double)f[j] * (double)f[j];
-      st_vec<T, V>(row + i, x);
+        for (int j = 0; j < V; ++j) acc += (double)f[j] * (double)f[j];
+      }
+    } else {
+      for (int i = threadIdx.x * V; i < d; i += step) {
+        const Vec<T, V> x = ld_vec<T, V>(hr + i);
+        float f[V];
+        vec_to_f32(x, f);
+#pragma unroll
+        for (int j = 0; j < V; ++j) acc += (double)f[j] * (double)f[j];
+        st_vec<T, V>(row + i, x);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -90,7 +107,7 @@ __global__ void __launch_bounds__(256) rmsnorm_router_kernel(const T* __restrict
     __syncthreads();
     const float r = r_sh;
     const bool store = (blockIdx.y == 0) && xn != nullptr;
-    for (int i = threadIdx.x * V; i < d; i += blockDim.x * V) {
+    for (int i = threadIdx.x * V; i < d; i += step) {
       float f[V], wf[V];
       vec_to_f32(ld_vec<T, V>(row + i), f);
       vec_to_f32(ld_vec<T, V>(w + i), wf);
@@ -126,7 +143,8 @@ __global__ void __launch_bounds__(256) rmsnorm_router_kernel(const T* __restrict
 //   score = softmax(logits) in fp32; key = fl32(score + bias);
 //   k rounds of a warp arg-max on key (equal keys: lower expert wins);
 //   gate_j = score_j / sum of the chosen scores.
-// counts: per-block shared histogram, added to the global one at the end.
+// counts: per-block shared histogram, added to the global one at the end
+// (skipped when counts is null).
 // ---------------------------------------------------------------------------
 template <int EPL>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits,
@@ -134,8 +152,10 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
                                                    int32_t* __restrict__ topk_idx, float* __restrict__ topk_gate,
                                                    int32_t* __restrict__ counts, int n, int E, int k) {
   extern __shared__ int32_t hist[];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
-  __syncthreads();
+  if (counts != nullptr) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+  }
   const int lane = lane_id();
   const int warps = blockDim.x >> 5;
   for (int t = blockIdx.x * warps + warp_id(); t < n; t += gridDim.x * warps) {
@@ -207,9 +227,10 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     if (lane < k) {
       topk_idx[(size_t)t * k + lane] = my_idx;
       topk_gate[(size_t)t * k + lane] = __fdiv_rn(my_score, chosen_sum);
-      atomicAdd(&hist[my_idx], 1);
+      if (counts != nullptr) atomicAdd(&hist[my_idx], 1);
     }
   }
+  if (counts == nullptr) return;
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)
     if (hist[e]) atomicAdd(&counts[e], hist[e]);
@@ -303,12 +324,12 @@ moe_status launch_rmsnorm_router(int dtype, const void* h, const void* norm_w, c
 
 moe_status launch_topk(const float* logits, const float* bias, float* scores, int32_t* topk_idx,
                        float* topk_gate, int32_t* counts, int n, int e, int k, cudaStream_t s) {
-  if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * e, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (counts != nullptr && cudaMemsetAsync(counts, 0, sizeof(int32_t) * e, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (n == 0) return MOE_OK;
   const int warps = 8;
   int blocks = (n + warps - 1) / warps;
   if (blocks > sm_count() * 8) blocks = sm_count() * 8;
-  size_t smem = sizeof(int32_t) * e;
+  size_t smem = counts != nullptr ? sizeof(int32_t) * e : 0;
   int epl = (e + 31) / 32;
 #define MOE_TOPK(EPL) \
   moe::topk_kernel<EPL><<<blocks, warps * 32, smem, s>>>(logits, bias, scores, topk_idx, topk_gate, counts, n, e, k)
