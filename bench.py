@@ -15,6 +15,10 @@ max over ranks and the value counts the tokens of all ranks.
 
 --impl reference times the CPU oracle (plain float64 numpy) on a bounded
 sample of the same workload on the host cores; rank 0 alone runs it.
+
+--library-baseline times the routed experts' FFN (gate/up, SwiGLU, down) of
+the workload through moe_expert_ffn against torch's grouped GEMM on the same
+row counts, one JSON line; it is context for the roofline, not the bench line.
 """
 from __future__ import annotations
 
@@ -325,9 +329,11 @@ def run_native(args):
                     "peak_kind": f"HBM copy, {peaks['source']}", "algorithmic_bytes": fb["gate_up_bytes"],
                     "touched_experts": fb["touched_experts"]}
         # library kernels per step: RMSNorm(+router), [router GEMM], top-k, 3 permute
-        # kernels, gather, 2 routed GEMMs, [2 shared GEMMs], combine
+        # kernels, row scatter, 2 routed GEMMs, [2 shared GEMMs unless the shared
+        # expert is folded into the routed ones], combine
         router_tc = cfg.dtype == "bf16" and cfg.n_experts >= 64 and cfg.n_tokens >= 512
-        launches = 1 + int(router_tc) + 1 + 3 + 1 + 2 + (2 if cfg.d_ff_shared > 0 else 0) + 1
+        shared_launches = 2 if cfg.d_ff_shared > 0 and not fb["shared_folded"] else 0
+        launches = 1 + int(router_tc) + 1 + 3 + 1 + 2 + shared_launches + 1
         line = {
             "metric": METRIC, "value": round(whole_job_tokens_per_s(cfg.n_tokens, world, ms), 1), "unit": UNIT,
             "n_gpus": world,
@@ -442,6 +448,94 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_library_baseline(args):
+    """The routed experts' FFN of the workload (its real per-expert row counts,
+    random bf16 rows) through moe_expert_ffn, against torch's grouped GEMM
+    (torch._grouped_mm) doing the same two projections, arms interleaved in one
+    process.  Context for the roofline figures, not a bench line of the layer."""
+    import numpy as np
+    import torch
+
+    import moe_inputs as mi
+    import sparse_mixture_experts_rmsnorm_b200 as moe
+
+    torch.cuda.set_device(0)
+    cfg = workload(args)
+    if cfg.dtype != "bf16":
+        print(json.dumps({"impl": "library-baseline", "unavailable": "torch._grouped_mm takes bf16 only"}))
+        return
+    lc = moe.Config(cfg.n_tokens, cfg.d_model, cfg.n_experts, cfg.top_k, cfg.d_ff, cfg.d_ff_shared, cfg.dtype,
+                    cfg.rms_eps, cfg.capacity_factor)
+    w = mi.device_tensors(cfg)
+    weights = {n: w[n] for n in ("norm_w", "w_router", "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down")
+               if n in w}
+    E, d, H = cfg.n_experts, cfg.d_model, cfg.d_ff
+    offsets = torch.zeros(E + 1, dtype=torch.int32, device="cuda")
+    ws = moe.workspace(lc)
+    moe.moe_layer_forward(lc, weights, w["h"], w["bias"], torch.empty_like(w["h"]), ws, routing={"offsets": offsets})
+    torch.cuda.synchronize()
+    R = int(offsets[-1])
+    gen = torch.Generator(device="cuda").manual_seed(0)
+    x = torch.randn(R, d, device="cuda", generator=gen).to(torch.bfloat16)
+    ffn_cfg = moe.Config(R, d, E, 1, H, 0, "bf16")
+    ffn_ws = moe.workspace(ffn_cfg)
+    y = torch.empty(R, d, dtype=torch.bfloat16, device="cuda")
+    wgu_t = torch.cat([w["w_gate"], w["w_up"]], dim=1).transpose(1, 2)  # [E][d][2H], K-major
+    wd_t = w["w_down"].transpose(1, 2)                                    # [E][H][d]
+    ends = offsets[1:].contiguous()
+    act = torch.randn(R, H, device="cuda", generator=gen).to(torch.bfloat16)
+
+    def ours():
+        moe.moe_expert_ffn(ffn_cfg, E, offsets, R, x, w["w_gate"], w["w_up"], w["w_down"], H, y, ffn_ws)
+
+    def torch_ffn():
+        t = torch._grouped_mm(x, wgu_t, offs=ends)
+        return torch._grouped_mm(torch.nn.functional.silu(t[:, :H]) * t[:, H:], wd_t, offs=ends)
+
+    def torch_gemms():
+        torch._grouped_mm(x, wgu_t, offs=ends)
+        torch._grouped_mm(act, wd_t, offs=ends)
+
+    arms = {"ours_ffn": ours}
+    note = None
+    try:
+        ref = torch_ffn()
+        torch.cuda.synchronize()
+        arms.update(torch_grouped_mm_ffn=torch_ffn, torch_grouped_mm_gemms_only=torch_gemms)
+    except Exception as ex:  # noqa: BLE001 - reported, not hidden
+        ref, note = None, f"torch._grouped_mm unavailable: {type(ex).__name__}: {str(ex)[:160]}"
+    iters = max(3, args.steps // 20)
+
+    def timed(fn):
+        s = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        fn()
+        e0.record(s)
+        for _ in range(iters):
+            fn()
+        e1.record(s)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / iters
+
+    times = {k: [] for k in arms}
+    order = list(arms)
+    for r in range(max(3, args.warmup)):
+        for k in (order if r % 2 == 0 else order[::-1]):
+            times[k].append(timed(arms[k]))
+    flops = 2.0 * R * d * 2 * H + 2.0 * R * H * d
+    line = {"impl": "library-baseline", "workload": cfg.name, "rows": R, "groups": E, "flop_per_call": flops,
+            "note": note}
+    for k, v in times.items():
+        ms = float(np.median(v))
+        line[k] = {"ms": round(ms, 4), "tflops": round(flops / ms / 1e9, 1)}
+    if ref is not None:
+        ours()
+        torch.cuda.synchronize()
+        diff = (y.float() - ref.float()).pow(2).mean().sqrt() / ref.float().pow(2).mean().sqrt()
+        line["rel_rms_diff_vs_torch"] = float(diff)
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -450,6 +544,8 @@ def main():
     ap.add_argument("--workload", default="mixtral_bf16")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--library-baseline", action="store_true",
+                    help="time the routed experts' FFN against torch._grouped_mm instead of the layer")
     ap.add_argument("--set", action="append", metavar="KEY=VALUE",
                     help="override a workload field, e.g. --set n_experts=32 --set n_tokens=1024")
     args = ap.parse_args()
@@ -457,6 +553,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         run_reference(args)
+    elif args.library_baseline:
+        run_library_baseline(args)
     else:
         run_native(args)
 

@@ -43,10 +43,12 @@ moe_status launch_permute(const int32_t* topk_idx, int n, int k, int e, int cap,
                           int32_t* offsets, int32_t* slot_row, int32_t* row_token, cudaStream_t s,
                           int32_t* offsets_ext = nullptr, int extra = 0, int32_t* counts = nullptr);
 
-// a5: x_perm[r] = xn[row_token[r]] for r < R = offsets[e] (device count),
-// and x_perm[R + t] = xn[t] for t < shared_rows (the folded shared expert).
-moe_status launch_gather(int dtype, const void* xn, const int32_t* row_token, const int32_t* offsets, int e,
-                         void* x_perm, int max_rows, int d, cudaStream_t s, int shared_rows = 0);
+// a5: x_perm[slot_row[t * k + j]] = xn[t] for every kept slot (that is,
+// x_perm[r] = xn[row_token[r]] for r < R = offsets[e], a device count), and
+// x_perm[R + t] = xn[t] for t < shared_rows (the folded shared expert).
+// Token order: each xn row is read once.  k <= 32.
+moe_status launch_gather(int dtype, const void* xn, const int32_t* slot_row, const int32_t* offsets, int e, int n,
+                         int k, void* x_perm, int d, cudaStream_t s, int shared_rows = 0);
 
 // a9: out = h + sum_j gate_j * y_perm[slot_row] (+ y_shared).  With
 // shared_offsets != nullptr the shared rows are y_perm rows from

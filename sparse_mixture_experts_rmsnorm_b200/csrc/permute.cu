@@ -20,8 +20,8 @@
 // expert into hist[e][chunk]; (2) one block scans each expert's row of hist
 // (giving every chunk the rank of its first slot within the expert) and
 // forms the kept counts and offsets; (3) the chunk warps recompute their
-// in-chunk ranks and write slot_row / row_token; (4) the gather copies rows
-// with 16-byte loads.
+// in-chunk ranks and write slot_row / row_token; (4) the gather copies each
+// token's row to its kept slots with 16-byte accesses.
 #include "moe_common.cuh"
 #include "moe_kernels.h"
 
@@ -171,21 +171,36 @@ __global__ void __launch_bounds__(kPermWarps * 32) chunk_scatter_kernel(
   });
 }
 
-// a5: x_perm[r] = xn[row_token[r]] for r < R = offsets[E], then
-// x_perm[R + t] = xn[t] for t < shared_rows.  One block per row,
-// grid-stride; VEC elements per 16-byte access when the row allows it.
+// a5 in token order: token t's row of xn is read once and written to each
+// of its kept slots, x_perm[slot_row[t * k + j]] = xn[t], and, with
+// shared_rows > 0, to x_perm[R + t] (R = offsets[E]) for the folded shared
+// expert.  Every x_perm row r < R has exactly one kept slot pointing at it,
+// so this writes the same x_perm as reading x_perm[r] = xn[row_token[r]],
+// while each xn row crosses HBM once instead of once per slot.  One block
+// per token (grid-stride); VEC elements per 16-byte access when the row
+// allows it.
 template <typename V>
-__global__ void __launch_bounds__(128) gather_rows_kernel(const V* __restrict__ xn,
-                                                          const int32_t* __restrict__ row_token,
-                                                          const int32_t* __restrict__ offsets, int E,
-                                                          V* __restrict__ x_perm, int row_vecs, int shared_rows) {
+__global__ void __launch_bounds__(128) scatter_rows_kernel(const V* __restrict__ xn,
+                                                           const int32_t* __restrict__ slot_row,
+                                                           const int32_t* __restrict__ offsets, int E, int n, int k,
+                                                           V* __restrict__ x_perm, int row_vecs, int shared_rows) {
+  __shared__ int32_t dst[33];
   const int routed = offsets[E];
-  const int rows = routed + shared_rows;
-  for (int r = blockIdx.x; r < rows; r += gridDim.x) {
-    const V* src = xn + (size_t)(r < routed ? row_token[r] : r - routed) * row_vecs;
-    V* dst = x_perm + (size_t)r * row_vecs;
+  const int nd = k + (shared_rows > 0 ? 1 : 0);
+  for (int t = blockIdx.x; t < n; t += gridDim.x) {
+    if (threadIdx.x < k) dst[threadIdx.x] = slot_row[(size_t)t * k + threadIdx.x];
+    if (threadIdx.x == 0 && shared_rows > 0) dst[k] = t < shared_rows ? routed + t : -1;
+    __syncthreads();
+    const V* src = xn + (size_t)t * row_vecs;
 #pragma unroll 4
-    for (int i = threadIdx.x; i < row_vecs; i += blockDim.x) dst[i] = src[i];
+    for (int i = threadIdx.x; i < row_vecs; i += blockDim.x) {
+      const V v = src[i];
+      for (int j = 0; j < nd; ++j) {
+        const int r = dst[j];
+        if (r >= 0) x_perm[(size_t)r * row_vecs + i] = v;
+      }
+    }
+    __syncthreads();
   }
 }
 
@@ -219,22 +234,22 @@ moe_status launch_permute(const int32_t* topk_idx, int n, int k, int e, int cap,
   return launch_status();
 }
 
-moe_status launch_gather(int dtype, const void* xn, const int32_t* row_token, const int32_t* offsets, int e,
-                         void* x_perm, int max_rows, int d, cudaStream_t s, int shared_rows) {
-  max_rows += shared_rows;
-  if (max_rows == 0) return MOE_OK;
+moe_status launch_gather(int dtype, const void* xn, const int32_t* slot_row, const int32_t* offsets, int e, int n,
+                         int k, void* x_perm, int d, cudaStream_t s, int shared_rows) {
+  if (n == 0) return MOE_OK;
+  if (k > 32) return MOE_ERR_UNSUPPORTED;
   const size_t row_bytes = (size_t)d * (dtype == MOE_BF16 ? 2 : 4);
-  int grid = max_rows < sm_count() * 16 ? max_rows : sm_count() * 16;
+  int grid = n < sm_count() * 16 ? n : sm_count() * 16;
   const uintptr_t addr = (uintptr_t)xn | (uintptr_t)x_perm;
   if (row_bytes % 16 == 0 && addr % 16 == 0)
-    moe::gather_rows_kernel<uint4><<<grid, 128, 0, s>>>((const uint4*)xn, row_token, offsets, e, (uint4*)x_perm,
-                                                        (int)(row_bytes / 16), shared_rows);
+    moe::scatter_rows_kernel<uint4><<<grid, 128, 0, s>>>((const uint4*)xn, slot_row, offsets, e, n, k,
+                                                         (uint4*)x_perm, (int)(row_bytes / 16), shared_rows);
   else if (row_bytes % 4 == 0 && addr % 4 == 0)
-    moe::gather_rows_kernel<uint32_t><<<grid, 128, 0, s>>>((const uint32_t*)xn, row_token, offsets, e,
-                                                           (uint32_t*)x_perm, (int)(row_bytes / 4), shared_rows);
+    moe::scatter_rows_kernel<uint32_t><<<grid, 128, 0, s>>>((const uint32_t*)xn, slot_row, offsets, e, n, k,
+                                                            (uint32_t*)x_perm, (int)(row_bytes / 4), shared_rows);
   else
-    moe::gather_rows_kernel<uint16_t><<<grid, 128, 0, s>>>((const uint16_t*)xn, row_token, offsets, e,
-                                                           (uint16_t*)x_perm, (int)(row_bytes / 2), shared_rows);
+    moe::scatter_rows_kernel<uint16_t><<<grid, 128, 0, s>>>((const uint16_t*)xn, slot_row, offsets, e, n, k,
+                                                            (uint16_t*)x_perm, (int)(row_bytes / 2), shared_rows);
   return launch_status();
 }
 

@@ -69,11 +69,10 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
   moe_status st = hist_address(&hist);
   if (st != MOE_OK) return st;
   const int64_t cap = capacity_of(cfg);
-  int64_t rows = slots;
-  if (cap >= 0 && (int64_t)cfg->n_experts * cap < rows) rows = (int64_t)cfg->n_experts * cap;
   cudaStream_t s = (cudaStream_t)stream;
   st = launch_permute(topk_idx, cfg->n_tokens, cfg->top_k, cfg->n_experts, (int)cap, hist, offsets, slot_row,
                       row_token, s);
   if (st != MOE_OK) return st;
-  return launch_gather(cfg->dtype, xn, row_token, offsets, cfg->n_experts, x_perm, (int)rows, cfg->d_model, s);
+  return launch_gather(cfg->dtype, xn, slot_row, offsets, cfg->n_experts, cfg->n_tokens, cfg->top_k, x_perm,
+                       cfg->d_model, s);
 }
