@@ -115,8 +115,8 @@ const char* moe_version(void);
  * activations [max(R*H, N*Hs)] and expert outputs y_perm [R][d], y_shared
  * [N][d], where R = N*k, or min(N*k, E*cap) with a capacity.  When the
  * shared expert is as wide as the routed ones (bf16, Hs == H) it runs as one
- * more group of the routed expert GEMMs: x_perm, act and y_perm then hold
- * R + N rows and there is no separate y_shared. */
+ * more group of the routed expert GEMMs, reading its input rows from xn:
+ * act and y_perm then hold R + N rows and there is no separate y_shared. */
 size_t moe_workspace_size(const moe_config* cfg);
 
 /* Zero the workspace header (the device error word).  Call once after

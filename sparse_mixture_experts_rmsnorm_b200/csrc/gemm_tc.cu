@@ -32,6 +32,8 @@
 // its copies and MMAs (again with a bound), frees its TMEM and returns.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 #include "tcgen05.cuh"
 
 namespace moe {
@@ -49,7 +51,8 @@ template <int EPI>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                    const __grid_constant__ CUtensorMap map_b2, const __grid_constant__ CUtensorMap map_sb,
-                   const __grid_constant__ CUtensorMap map_sb2, const TcArgs args) {
+                   const __grid_constant__ CUtensorMap map_sb2, const __grid_constant__ CUtensorMap map_sa,
+                   const TcArgs args) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[TC_STAGES];
   __shared__ __align__(8) uint64_t empty_bar[TC_STAGES];
@@ -102,6 +105,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tma_prefetch_map(&map_a);
       tma_prefetch_map(&map_b);
       tma_prefetch_map(&map_b2);
+      if (args.shared_a) tma_prefetch_map(&map_sa);
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
@@ -113,6 +117,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const CUtensorMap* mb = sh ? &map_sb : &map_b;
         const CUtensorMap* mb2 = sh ? &map_sb2 : &map_b2;
         const int brow = (sh ? 0 : tl.group * args.nout) + tl.n0;
+        // ... and, when given its own A map, reads its rows from there
+        const bool sa_own = sh && args.shared_a;
+        const CUtensorMap* ma = sa_own ? &map_sa : &map_a;
+        const int arow = sa_own ? tl.row0 - offs_sh[tl.group] : tl.row0;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
                                  SITE_EMPTY)) {
@@ -121,7 +129,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
           const uint32_t sa = smem_base + stage * TC_STAGE_BYTES;
           mbar_arrive_expect_tx(&full_bar[stage], TC_STAGE_BYTES);
-          tma_load_2d(sa, &map_a, &full_bar[stage], kb * TC_BK, tl.row0);
+          tma_load_2d(sa, ma, &full_bar[stage], kb * TC_BK, arow);
           if (EPI == moe_host::EPI_SWIGLU) {
             tma_load_2d(sa + TC_A_BYTES, mb, &full_bar[stage], kb * TC_BK, brow);
             tma_load_2d(sa + TC_A_BYTES + TC_B_HALF_BYTES, mb2, &full_bar[stage], kb * TC_BK, brow);
@@ -279,8 +287,8 @@ bool make_tc_map(CUtensorMap* m, const void* base, int64_t rows, int k) {
 
 template <int EPI>
 static moe_status launch_tc_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
-                              const CUtensorMap& msb, const CUtensorMap& msb2, const moe::TcArgs& args, int grid,
-                              cudaStream_t s) {
+                              const CUtensorMap& msb, const CUtensorMap& msb2, const CUtensorMap& msa,
+                              const moe::TcArgs& args, int grid, cudaStream_t s) {
   static bool attr_done[64] = {};
   int dev = current_device();
   if (dev < 64 && !attr_done[dev]) {
@@ -289,25 +297,30 @@ static moe_status launch_tc_t(const CUtensorMap& ma, const CUtensorMap& mb, cons
       return MOE_ERR_CUDA;
     attr_done[dev] = true;
   }
-  moe::gemm_tc_kernel<EPI><<<grid, moe::TC_THREADS, moe::TC_SMEM_BYTES, s>>>(ma, mb, mb2, msb, msb2, args);
+  moe::gemm_tc_kernel<EPI><<<grid, moe::TC_THREADS, moe::TC_SMEM_BYTES, s>>>(ma, mb, mb2, msb, msb2, msa, args);
   return launch_status();
 }
 
 moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2, const int32_t* offsets,
                           int groups, int max_rows, int nout, int k, void* c, int ldc, int32_t* hdr, cudaStream_t s,
-                          const void* sb, const void* sb2) {
+                          const void* sb, const void* sb2, const void* sa, int sa_rows) {
   if (max_rows == 0 || nout == 0 || groups == 0) return MOE_OK;
   if (groups > moe::TC_MAX_GROUPS || (k % 8) != 0) return MOE_ERR_UNSUPPORTED;
   if (((uintptr_t)a | (uintptr_t)b | (uintptr_t)(b2 ? b2 : b) | (uintptr_t)(sb ? sb : b) |
-       (uintptr_t)(sb2 ? sb2 : b)) % 16 != 0)
+       (uintptr_t)(sb2 ? sb2 : b) | (uintptr_t)(sa ? sa : a)) % 16 != 0)
     return MOE_ERR_UNSUPPORTED;
-  CUtensorMap ma, mb, mb2, msb, msb2;
+  CUtensorMap ma, mb, mb2, msb, msb2, msa;
   // the routed weights hold one [nout][k] block per routed group only: a
   // folded shared expert (the last group) has its own tensor, so the map must
   // end at the routed allocation for TMA to zero-fill past it
   const int routed_groups = (sb != nullptr && offsets) ? groups - 1 : groups;
   const int64_t b_rows = (int64_t)routed_groups * nout;
-  if (!make_tc_map(&ma, a, max_rows, k) || !make_tc_map(&mb, b, b_rows, k)) return MOE_ERR_CUDA;
+  // with its own A map the shared group's rows are not in `a`, which then
+  // holds the routed rows only
+  const bool shared_a = sb != nullptr && offsets && sa != nullptr && sa_rows > 0;
+  // (no routed rows at all: the map is never read, but must hold a row)
+  const int64_t a_rows = shared_a ? std::max<int64_t>((int64_t)max_rows - sa_rows, 1) : max_rows;
+  if (!make_tc_map(&ma, a, a_rows, k) || !make_tc_map(&mb, b, b_rows, k)) return MOE_ERR_CUDA;
   if (epi == EPI_SWIGLU) {
     if (!make_tc_map(&mb2, b2, b_rows, k)) return MOE_ERR_CUDA;
   } else {
@@ -325,6 +338,12 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
     msb = mb;
     msb2 = mb2;
   }
+  // the folded shared expert's input rows, when they are not in `a`
+  if (shared_a) {
+    if (!make_tc_map(&msa, sa, sa_rows, k)) return MOE_ERR_CUDA;
+  } else {
+    msa = ma;
+  }
   moe::TcArgs args;
   args.offsets = offsets;
   args.groups = offsets ? groups : 1;
@@ -338,20 +357,21 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
   args.hdr = hdr;
   args.wait_ns = wait_limit_ns();
   args.shared_group = (sb != nullptr && offsets) ? groups - 1 : -1;
+  args.shared_a = shared_a ? 1 : 0;
   const int rows_per_group = max_rows / (offsets ? groups : 1);
   const int mode = tc_pairing();
   // Measured on B200: SM pairs help the plain-store epilogue of large groups
   // (down projection, router) by a few percent; for the SwiGLU projection the
   // extra padding of 256-row tiles outweighs the saved operand traffic.
   if (mode == 2 || (mode == 0 && rows_per_group >= 512 && epi != EPI_SWIGLU))
-    return launch_gemm_tc2(epi, ma, mb, mb2, msb, msb2, args, max_rows, offsets ? groups : 0, s);
+    return launch_gemm_tc2(epi, ma, mb, mb2, msb, msb2, msa, args, max_rows, offsets ? groups : 0, s);
   // Upper bound on the number of tiles; the exact count lives on the device.
   const int64_t m_tiles = (int64_t)(max_rows + moe::TC_BM - 1) / moe::TC_BM + (offsets ? groups : 0);
   const int64_t bound = m_tiles * args.n_tiles;
   const int grid = (int)(bound < sm_count() ? bound : sm_count());
-  if (epi == EPI_SWIGLU) return launch_tc_t<EPI_SWIGLU>(ma, mb, mb2, msb, msb2, args, grid, s);
-  if (epi == EPI_STORE) return launch_tc_t<EPI_STORE>(ma, mb, mb2, msb, msb2, args, grid, s);
-  return launch_tc_t<EPI_F32>(ma, mb, mb2, msb, msb2, args, grid, s);
+  if (epi == EPI_SWIGLU) return launch_tc_t<EPI_SWIGLU>(ma, mb, mb2, msb, msb2, msa, args, grid, s);
+  if (epi == EPI_STORE) return launch_tc_t<EPI_STORE>(ma, mb, mb2, msb, msb2, msa, args, grid, s);
+  return launch_tc_t<EPI_F32>(ma, mb, mb2, msb, msb2, msa, args, grid, s);
 }
 
 static int g_pairing = 0;

@@ -98,7 +98,8 @@ template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                     const __grid_constant__ CUtensorMap map_b2, const __grid_constant__ CUtensorMap map_sb,
-                    const __grid_constant__ CUtensorMap map_sb2, const TcArgs args) {
+                    const __grid_constant__ CUtensorMap map_sb2, const __grid_constant__ CUtensorMap map_sa,
+                    const TcArgs args) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[P_STAGES];   // used in the even CTA
   __shared__ __align__(8) uint64_t empty_bar[P_STAGES];
@@ -152,6 +153,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     // ======================= TMA producer (both CTAs) =======================
     if (lane == 0) {
       tma_prefetch_map(&map_a);
+      if (args.shared_a) tma_prefetch_map(&map_sa);
       const bool second = rank == 1 && EPI == moe_host::EPI_SWIGLU;  // the up half of a SwiGLU tile
       tma_prefetch_map(second ? &map_b2 : &map_b);
       int stage = 0;
@@ -162,7 +164,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
         const Tile tl = decode_tile<P_BM>(t, prefix_sh, offs_sh, G, args.out_cols);
         const bool sh = tl.group == args.shared_group;  // the folded shared expert has its own weights
         const CUtensorMap* bmap = sh ? (second ? &map_sb2 : &map_sb) : (second ? &map_b2 : &map_b);
-        const int a_row = tl.row0 + (int)rank * 128;
+        // the folded shared expert's rows may come from their own A map, from row 0
+        const bool sa_own = sh && args.shared_a;
+        const CUtensorMap* amap = sa_own ? &map_sa : &map_a;
+        const int a_row = (sa_own ? tl.row0 - offs_sh[tl.group] : tl.row0) + (int)rank * 128;
         const int b_row = (sh ? 0 : tl.group * args.nout) + tl.n0 + (EPI == moe_host::EPI_SWIGLU ? 0 : (int)rank * 128);
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
@@ -173,7 +178,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
           const uint32_t sa = smem_base + stage * P_STAGE_BYTES;
           const uint32_t full_leader = map_to_rank(&full_bar[stage], 0);
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * P_STAGE_BYTES);
-          tma_load_2d_pair(sa, &map_a, full_leader, kb * TC_BK, a_row);
+          tma_load_2d_pair(sa, amap, full_leader, kb * TC_BK, a_row);
           tma_load_2d_pair(sa + P_A_BYTES, bmap, full_leader, kb * TC_BK, b_row);
           ++issued;
           if (++stage == P_STAGES) {
@@ -306,8 +311,8 @@ static int resident_pairs() {
 
 template <int EPI>
 static moe_status launch_tc2_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
-                               const CUtensorMap& msb, const CUtensorMap& msb2, const moe::TcArgs& args,
-                               int64_t pair_bound, cudaStream_t s) {
+                               const CUtensorMap& msb, const CUtensorMap& msb2, const CUtensorMap& msa,
+                               const moe::TcArgs& args, int64_t pair_bound, cudaStream_t s) {
   static bool attr_done[64] = {};
   int dev = current_device();
   if (dev < 64 && !attr_done[dev]) {
@@ -318,20 +323,20 @@ static moe_status launch_tc2_t(const CUtensorMap& ma, const CUtensorMap& mb, con
   }
   const int64_t pairs = pair_bound < resident_pairs<EPI>() ? pair_bound : resident_pairs<EPI>();
   moe::gemm_tc2_kernel<EPI><<<(unsigned)(2 * pairs), moe::P_THREADS, moe::P_SMEM_BYTES, s>>>(ma, mb, mb2, msb, msb2,
-                                                                                          args);
+                                                                                          msa, args);
   return launch_status();
 }
 
 // Launch of the SM-pair kernel; maps and arguments come from launch_gemm_tc.
 moe_status launch_gemm_tc2(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
-                           const CUtensorMap& msb, const CUtensorMap& msb2, const moe::TcArgs& args, int64_t max_rows,
-                           int groups_bound, cudaStream_t s) {
+                           const CUtensorMap& msb, const CUtensorMap& msb2, const CUtensorMap& msa,
+                           const moe::TcArgs& args, int64_t max_rows, int groups_bound, cudaStream_t s) {
   // upper bound on the pair tiles; the exact count lives on the device
   const int64_t m_pairs = (max_rows + moe::P_BM - 1) / moe::P_BM + groups_bound;
   const int64_t bound = m_pairs * args.n_tiles;
-  if (epi == EPI_SWIGLU) return launch_tc2_t<EPI_SWIGLU>(ma, mb, mb2, msb, msb2, args, bound, s);
-  if (epi == EPI_STORE) return launch_tc2_t<EPI_STORE>(ma, mb, mb2, msb, msb2, args, bound, s);
-  return launch_tc2_t<EPI_F32>(ma, mb, mb2, msb, msb2, args, bound, s);
+  if (epi == EPI_SWIGLU) return launch_tc2_t<EPI_SWIGLU>(ma, mb, mb2, msb, msb2, msa, args, bound, s);
+  if (epi == EPI_STORE) return launch_tc2_t<EPI_STORE>(ma, mb, mb2, msb, msb2, msa, args, bound, s);
+  return launch_tc2_t<EPI_F32>(ma, mb, mb2, msb, msb2, msa, args, bound, s);
 }
 
 }  // namespace moe_host

@@ -53,7 +53,8 @@ static Layout layout_of(const moe_config* c) {
   if (cap >= 0 && E * cap < R) R = E * cap;
   L.rows = R;
   // bf16 layers with a shared expert as wide as the routed ones fold it into
-  // the routed GEMMs: its N rows follow the R routed rows in x_perm, act and y_perm
+  // the routed GEMMs: its N rows follow the R routed rows in act and y_perm,
+  // and the gate/up GEMM reads its input rows straight from xn
   L.fold = c->dtype == MOE_BF16 && c->d_ff_shared > 0 && c->d_ff_shared == c->d_ff &&
            c->n_experts < moe::TC_MAX_GROUPS;
   const int64_t Rx = R + (L.fold ? N : 0);
@@ -76,7 +77,7 @@ static Layout layout_of(const moe_config* c) {
   L.slot_row = take(N * k * 4);
   L.row_token = take(N * k * 4);
   L.hist = take(permute_hist_ints(N * k, (int)E) * 4);
-  L.x_perm = take(Rx * d * es);
+  L.x_perm = take(R * d * es);
   L.act = take(L.act_elems * es);
   L.y_perm = take(Rx * d * es);
   L.y_shared = take(c->d_ff_shared > 0 && !L.fold ? N * d * es : 0);
@@ -305,12 +306,11 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const 
     int32_t* offs_ext = (int32_t*)wsp(ws, L.offsets_ext);
     MOE_TRY(launch_permute(idx, N, cfg->top_k, cfg->n_experts, (int)capacity_of(cfg), (int32_t*)wsp(ws, L.hist),
                            offsets, slot_row, row_token, s, offs_ext, N, counts));
-    MOE_TRY(launch_gather(cfg->dtype, xn, slot_row, offsets, cfg->n_experts, N, cfg->top_k, x_perm, cfg->d_model, s,
-                          N));
+    MOE_TRY(launch_gather(cfg->dtype, xn, slot_row, offsets, cfg->n_experts, N, cfg->top_k, x_perm, cfg->d_model, s));
     MOE_TRY(mark(trace ? trace->permuted : nullptr));
     if (N > 0) {
       MOE_TRY(launch_gemm_tc(EPI_SWIGLU, x_perm, w->w_gate, w->w_up, offs_ext, cfg->n_experts + 1, R + N, cfg->d_ff,
-                             cfg->d_model, act, cfg->d_ff, hdr, s, w->ws_gate, w->ws_up));
+                             cfg->d_model, act, cfg->d_ff, hdr, s, w->ws_gate, w->ws_up, xn, N));
       MOE_TRY(mark(trace ? trace->gate_up : nullptr));
       MOE_TRY(launch_gemm_tc(EPI_STORE, act, w->w_down, nullptr, offs_ext, cfg->n_experts + 1, R + N, cfg->d_model,
                              cfg->d_ff, y_perm, cfg->d_model, hdr, s, w->ws_down, nullptr));

@@ -78,9 +78,12 @@ moe_status launch_gemm_simt(int dtype, int epi, const void* a, const void* b, co
 //   hdr: workspace header that receives a device time-out, if any.
 //   sb, sb2 != nullptr: the last group is the shared expert, with its own
 //   [nout][k] weights sb (gate or down) and sb2 (up).
+//   sa != nullptr (with sb): that group's A rows are sa [sa_rows][k] instead
+//   of rows offsets[G-1].. of a.
 moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2, const int32_t* offsets,
                           int groups, int max_rows, int nout, int k, void* c, int ldc, int32_t* hdr, cudaStream_t s,
-                          const void* sb = nullptr, const void* sb2 = nullptr);
+                          const void* sb = nullptr, const void* sb2 = nullptr, const void* sa = nullptr,
+                          int sa_rows = 0);
 
 // A block that waits, with the bounded wait of the pipelined kernels, on a
 // barrier that nothing completes.

@@ -96,6 +96,7 @@ __global__ void __launch_bounds__(1024) hist_scan_kernel(int32_t* __restrict__ h
       }
 #pragma unroll
       for (int i = 0; i < kScanPer; ++i) {
+        if (c0 + 32 * i >= nchunks) break;  // uniform across the warp
         int32_t x = v[i];
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {

@@ -31,6 +31,7 @@ struct TcArgs {
   int32_t* hdr;
   uint64_t wait_ns;
   int shared_group;  // group whose weights come from the second map pair (-1: none)
+  int shared_a;      // 1: that group's A rows come from their own map, from row 0
 };
 
 // ---- PTX wrappers -----------------------------------------------------------
@@ -231,8 +232,8 @@ bool make_tc_map(CUtensorMap* m, const void* base, int64_t rows, int k);
 // The SM-pair kernel (gemm_tc2.cu) on maps and arguments prepared by
 // launch_gemm_tc; groups_bound = groups when offsets are given, else 0.
 moe_status launch_gemm_tc2(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
-                           const CUtensorMap& msb, const CUtensorMap& msb2, const moe::TcArgs& args, int64_t max_rows,
-                           int groups_bound, cudaStream_t s);
+                           const CUtensorMap& msb, const CUtensorMap& msb2, const CUtensorMap& msa,
+                           const moe::TcArgs& args, int64_t max_rows, int groups_bound, cudaStream_t s);
 
 // 0: choose per launch (SM pairs for the store / fp32 epilogues when the
 //    groups average >= 512 rows);

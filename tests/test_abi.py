@@ -66,9 +66,10 @@ def test_workspace_bytes_match_the_documented_regions():
     need32 = N * d * 4 + routing + 2 * R * d * 4 + max(R * H, N * Hs) * 4 + N * d * 4
     assert need32 <= moe.workspace_size(f) <= need32 + 64 * 1024
     # bf16 with a shared expert as wide as the routed ones: it is one more
-    # group of N rows in x_perm, act and y_perm, and there is no separate y_shared
+    # group of N rows in act and y_perm (its input rows are read from xn), and
+    # there is no separate y_shared
     g = _cfg(dtype="bf16", n_tokens=N, d_model=d, n_experts=E, top_k=k, d_ff=H, d_ff_shared=H)
-    need_f = N * d * 2 + routing + 2 * (R + N) * d * 2 + (R + N) * H * 2
+    need_f = N * d * 2 + routing + R * d * 2 + (R + N) * d * 2 + (R + N) * H * 2
     assert need_f <= moe.workspace_size(g) <= need_f + 64 * 1024
 
 

@@ -314,6 +314,8 @@ def test_device_wait_times_out_and_reports(torch_cuda):
     # shared expert as wide as the routed ones (it runs inside the routed GEMMs) plus drops
     dict(n_tokens=400, d_model=256, n_experts=8, top_k=2, d_ff=128, d_ff_shared=128, capacity_factor=0.8,
          skew=(2, 8.0, 2.5)),
+    # capacity 0: every routed slot dropped, the folded shared expert alone adds to h
+    dict(n_tokens=64, d_model=128, n_experts=16, top_k=2, d_ff=64, d_ff_shared=64, capacity_factor=0.05),
 ])
 def test_small_bf16_layer_every_output(torch_cuda, over):
     cfg = mi.LayerConfig(name="small", dtype="bf16", seed=4, **over)
@@ -330,6 +332,20 @@ def test_small_bf16_layer_every_output(torch_cuda, over):
     if cfg.d_ff_shared == 0 and dropped_all.size:
         np.testing.assert_array_equal(g["out"][dropped_all], ref["h"][dropped_all] if "h" in ref else
                                       mi.host_tensor(cfg, "h")[dropped_all])
+
+
+@pytest.mark.parametrize("mode", [1, 2])  # single-SM tiles, SM-pair tiles
+def test_folded_shared_expert_in_both_tilings(torch_cuda, gemm_tiling, mode):
+    # the shared expert runs as the last group of the routed GEMMs and reads
+    # its input rows from xn through its own tensor map, in either kernel
+    gemm_tiling(mode)
+    cfg = mi.LayerConfig(name="fold", dtype="bf16", seed=7, n_tokens=700, d_model=256, n_experts=8, top_k=2,
+                         d_ff=192, d_ff_shared=192)
+    g = run_gpu_layer(cfg)
+    ref = _full_oracle(cfg)
+    err = bf16_rel_rms_err(g["out"], ref["out64"])
+    print(f"folded shared expert, tiling {mode}: beyond-storage max err/rms {err:.3e}")
+    assert err <= BF16_REL_RMS, err
 
 
 # ----------------------------------------------------------------- the forward pass as a CUDA graph
