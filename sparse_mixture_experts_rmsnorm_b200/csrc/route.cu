@@ -22,8 +22,7 @@ namespace moe {
 // r = fl32(1 / sqrt(ms + eps)) is taken in fp64 and rounded once, then
 // xn = round(fl32(fl32(h * r) * w)), so the storage rounding is decided in fp32.
 //
-// One block per token (grid-stride), V elements per 16-byte access; the row
-// comes in with cp.async, all of its copies in flight at once.  The
+// One block per token (grid-stride), V elements per 16-byte access.  The
 // row is staged in shared memory in its own dtype; when `logits` is given, the
 // block's warps then take the router dot products of the rounded xn row
 // with experts [e0, e0 + epb) (e0 = blockIdx.y * epb), one expert per warp
@@ -72,28 +71,13 @@ __global__ void __launch_bounds__(256) rmsnorm_router_kernel(const T* __restrict
   for (int t = blockIdx.x; t < n; t += gridDim.x) {
     const T* hr = h + (size_t)t * d;
     double acc = 0.0;
-    if (V * sizeof(T) == 16) {
-      // every 16-byte copy of the row in flight at once (cp.async, no
-      // registers held); each thread then reads back the elements it copied,
-      // in increasing order
-      for (int i = threadIdx.x * V; i < d; i += step)
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(row + i)), "l"(hr + i) : "memory");
-      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-      for (int i = threadIdx.x * V; i < d; i += step) {
-        float f[V];
-        vec_to_f32(ld_vec<T, V>(row + i), f);
+    for (int i = threadIdx.x * V; i < d; i += step) {
+      const Vec<T, V> x = ld_vec<T, V>(hr + i);
+      float f[V];
+      vec_to_f32(x, f);
 #pragma unroll
-        for (int j = 0; j < V; ++j) acc += (double)f[j] * (double)f[j];
-      }
-    } else {
-      for (int i = threadIdx.x * V; i < d; i += step) {
-        const Vec<T, V> x = ld_vec<T, V>(hr + i);
-        float f[V];
-        vec_to_f32(x, f);
-#pragma unroll
-        for (int j = 0; j < V; ++j) acc += (double)f[j] * (double)f[j];
-        st_vec<T, V>(row + i, x);
-      }
+      for (int j = 0; j < V; ++j) acc += (double)f[j] * (double)f[j];
+      st_vec<T, V>(row + i, x);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
