@@ -172,6 +172,101 @@ __global__ void __launch_bounds__(kPermWarps * 32) chunk_scatter_kernel(
   });
 }
 
+// Kernels (1)-(3) in one block of 1024 threads, for up to 32 chunks when
+// the histogram and the per-warp running counts fit shared memory
+// (decode-sized and Mixtral-sized batches): warp w walks chunk w, the
+// histogram stays in shared memory, and the same scans and ranks as above
+// follow with block barriers instead of kernel boundaries.
+__global__ void __launch_bounds__(1024) permute_fused_kernel(const int32_t* __restrict__ idx, int64_t slots, int k,
+                                                             int E, int nchunks, int cap,
+                                                             int32_t* __restrict__ offsets,
+                                                             int32_t* __restrict__ offsets_ext, int extra,
+                                                             int32_t* __restrict__ counts,
+                                                             int32_t* __restrict__ slot_row,
+                                                             int32_t* __restrict__ row_token) {
+  extern __shared__ int32_t sm[];
+  int32_t* hist = sm;                         // [E][nchunks]
+  int32_t* run = sm + (size_t)E * nchunks + (size_t)warp_id() * E;  // this warp's running counts
+  __shared__ int32_t kept_sh[1024];
+  __shared__ int32_t offs_sh[1024];
+  __shared__ int32_t warp_sum[32];
+  const int lane = lane_id(), warp = warp_id();
+  const int c = warp;
+  for (int e = lane; e < E; e += 32) run[e] = 0;
+  __syncwarp();
+  if (c < nchunks) {
+    chunk_walk(idx, slots, c, run, [](int64_t, int, int) {});
+    for (int e = lane; e < E; e += 32) hist[e * nchunks + c] = run[e];
+  }
+  __syncthreads();
+  // exclusive scan of each expert's row over the chunks (nchunks <= 32)
+  for (int e = warp; e < E; e += 32) {
+    const int32_t v = lane < nchunks ? hist[e * nchunks + lane] : 0;
+    int32_t x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane < nchunks) hist[e * nchunks + lane] = x - v;
+    const int32_t total = __shfl_sync(0xffffffffu, x, 31);
+    if (lane == 0) {
+      kept_sh[e] = (cap >= 0 && total > cap) ? cap : total;
+      if (counts != nullptr) counts[e] = total;
+    }
+  }
+  __syncthreads();
+  const int tid = threadIdx.x;
+  const int32_t kv = (tid < E) ? kept_sh[tid] : 0;
+  int32_t x = kv;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sum[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = warp_sum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    warp_sum[lane] = w;
+  }
+  __syncthreads();
+  const int32_t excl = x - kv + (warp > 0 ? warp_sum[warp - 1] : 0);
+  if (tid < E) {
+    offs_sh[tid] = excl;
+    offsets[tid] = excl;
+    if (offsets_ext != nullptr) offsets_ext[tid] = excl;
+  }
+  if (tid == E - 1) {
+    offsets[E] = excl + kv;
+    if (offsets_ext != nullptr) {
+      offsets_ext[E] = excl + kv;
+      offsets_ext[E + 1] = excl + kv + extra;
+    }
+  }
+  __syncthreads();
+  // ranks: the chunk's first rank per expert plus the in-chunk rank
+  for (int e = lane; e < E; e += 32) run[e] = 0;
+  __syncwarp();
+  if (c < nchunks) {
+    chunk_walk(idx, slots, c, run, [&](int64_t s, int e, int r_in_chunk) {
+      const int32_t rank = hist[e * nchunks + c] + r_in_chunk;
+      if (cap < 0 || rank < cap) {
+        const int32_t row = offs_sh[e] + rank;
+        slot_row[s] = row;
+        row_token[row] = (int32_t)(s / k);
+      } else {
+        slot_row[s] = -1;
+      }
+    });
+  }
+}
+
 // a5 in token order: token t's row of xn is read once and written to each
 // of its kept slots, x_perm[slot_row[t * k + j]] = xn[t], and, with
 // shared_rows > 0, to x_perm[R + t] (R = offsets[E]) for the folded shared
@@ -225,6 +320,21 @@ moe_status launch_permute(const int32_t* topk_idx, int n, int k, int e, int cap,
       return MOE_ERR_CUDA;
     if (counts != nullptr && cudaMemsetAsync(counts, 0, sizeof(int32_t) * e, s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
+  }
+  // one block for small batches: histogram and running counts in shared memory
+  const size_t fused_smem = sizeof(int32_t) * (size_t)e * (size_t)(nch + 32);
+  if (nch <= 32 && fused_smem <= 96 * 1024) {
+    static bool attr_done[64] = {};
+    const int dev = current_device();
+    if (dev >= 64 || !attr_done[dev]) {
+      if (cudaFuncSetAttribute(moe::permute_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024) !=
+          cudaSuccess)
+        return MOE_ERR_CUDA;
+      if (dev < 64) attr_done[dev] = true;
+    }
+    moe::permute_fused_kernel<<<1, 1024, fused_smem, s>>>(topk_idx, slots, k, e, (int)nch, cap, offsets, offsets_ext,
+                                                          extra, counts, slot_row, row_token);
+    return launch_status();
   }
   const int blocks = (int)((nch + moe::kPermWarps - 1) / moe::kPermWarps);
   const size_t smem = sizeof(int32_t) * e * moe::kPermWarps;
