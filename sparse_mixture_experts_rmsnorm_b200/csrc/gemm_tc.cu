@@ -24,7 +24,9 @@
 // of the next.  A tile of at most 64 rows (a ragged expert's last tile, or
 // every tile of a decode step) runs as M = 64 MMAs; its accumulator keeps row
 // r in TMEM lane (r / 16) * 32 + r % 16, the first 16 lanes of each quarter.  For SwiGLU, B holds 128 gate rows then 128 up rows of the
-// same hidden units, so one N = 256 MMA produces both halves.
+// same hidden units, so one N = 256 MMA produces both halves.  A plain-
+// epilogue launch with too few tiles to fill the SMs (the router's logits)
+// uses 128-column tiles: one B box per stage and N = 128 MMAs.
 // Tiles are numbered group-major, then n-tile, then m-tile, so CTAs working
 // at the same time share weight tiles through L2.
 // Every mbarrier wait is bounded: on time-out the block records
@@ -128,14 +130,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             break;
           }
           const uint32_t sa = smem_base + stage * TC_STAGE_BYTES;
-          mbar_arrive_expect_tx(&full_bar[stage], TC_STAGE_BYTES);
+          const bool narrow = EPI != moe_host::EPI_SWIGLU && args.narrow;
+          mbar_arrive_expect_tx(&full_bar[stage], narrow ? TC_A_BYTES + TC_B_HALF_BYTES : TC_STAGE_BYTES);
           tma_load_2d(sa, ma, &full_bar[stage], kb * TC_BK, arow);
           if (EPI == moe_host::EPI_SWIGLU) {
             tma_load_2d(sa + TC_A_BYTES, mb, &full_bar[stage], kb * TC_BK, brow);
             tma_load_2d(sa + TC_A_BYTES + TC_B_HALF_BYTES, mb2, &full_bar[stage], kb * TC_BK, brow);
           } else {
             tma_load_2d(sa + TC_A_BYTES, mb, &full_bar[stage], kb * TC_BK, brow);
-            tma_load_2d(sa + TC_A_BYTES + TC_B_HALF_BYTES, mb, &full_bar[stage], kb * TC_BK, brow + 128);
+            if (!narrow)
+              tma_load_2d(sa + TC_A_BYTES + TC_B_HALF_BYTES, mb, &full_bar[stage], kb * TC_BK, brow + 128);
           }
           ++issued;
           if (++stage == TC_STAGES) {
@@ -159,7 +163,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   } else if (warp == 1) {
     // ======================= MMA issuer =======================
     if (lane == 0) {
-      constexpr uint32_t idesc = tc_idesc(TC_BM, TC_BN);
+      // 128-column tiles (plain epilogues with few tiles) run N = 128 MMAs
+      const int bn = (EPI != moe_host::EPI_SWIGLU && args.narrow) ? 128 : TC_BN;
+      const uint32_t idesc = tc_idesc(TC_BM, bn);
       int stage = 0;
       uint32_t phase = 0;
       int buf = 0;
@@ -168,7 +174,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
         const Tile tl = decode_tile<TC_BM>(t, prefix_sh, offs_sh, G, args.out_cols);
         // a tile of at most 64 rows runs as M = 64 MMAs (half the rows of work)
-        const uint32_t id = (tl.row_end - tl.row0 <= 64) ? tc_idesc(64, TC_BN) : idesc;
+        const uint32_t id = (tl.row_end - tl.row0 <= 64) ? tc_idesc(64, bn) : idesc;
         if (!mbar_wait_bounded(&tempty_bar[buf], bphase ^ 1u, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
                                SITE_TMEM_EMPTY))
           break;
@@ -224,7 +230,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       // 0..15 of each warp's quarter
       const bool half = tl.row_end - tl.row0 <= 64;
       const int row = half ? tl.row0 + quarter * 16 + (lane & 15) : tl.row0 + r_local;
-      epilogue_row<EPI>(args, tbase, row, row < tl.row_end && (!half || lane < 16), tl.n0);
+      epilogue_row<EPI>(args, tbase, row, row < tl.row_end && (!half || lane < 16), tl.n0, args.narrow ? 128 : 256);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty_bar[buf]);
@@ -352,6 +358,7 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
   args.K = k;
   args.out_cols = (epi == EPI_SWIGLU) ? 128 : moe::TC_BN;
   args.n_tiles = (nout + args.out_cols - 1) / args.out_cols;
+  args.narrow = 0;
   args.C = c;
   args.ldc = ldc;
   args.hdr = hdr;
@@ -360,13 +367,22 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
   args.shared_a = shared_a ? 1 : 0;
   const int rows_per_group = max_rows / (offsets ? groups : 1);
   const int mode = tc_pairing();
-  // Measured on B200: SM pairs help the plain-store epilogue of large groups
-  // (down projection, router) by a few percent; for the SwiGLU projection the
-  // extra padding of 256-row tiles outweighs the saved operand traffic.
-  if (mode == 2 || (mode == 0 && rows_per_group >= 512 && epi != EPI_SWIGLU))
-    return launch_gemm_tc2(epi, ma, mb, mb2, msb, msb2, msa, args, max_rows, offsets ? groups : 0, s);
   // Upper bound on the number of tiles; the exact count lives on the device.
   const int64_t m_tiles = (int64_t)(max_rows + moe::TC_BM - 1) / moe::TC_BM + (offsets ? groups : 0);
+  // A plain-epilogue launch that would leave more than half the SMs idle
+  // (the router's N x E logits: one 256-column tile per 128 rows) runs
+  // 128-column tiles on single SMs instead, twice as many.
+  const bool few = epi != EPI_SWIGLU && mode != 2 && nout > 128 && m_tiles * args.n_tiles < sm_count() / 2;
+  // Measured on B200: SM pairs help the plain-store epilogue of large groups
+  // (down projection) by a few percent; for the SwiGLU projection the extra
+  // padding of 256-row tiles outweighs the saved operand traffic.
+  if (mode == 2 || (mode == 0 && rows_per_group >= 512 && epi != EPI_SWIGLU && !few))
+    return launch_gemm_tc2(epi, ma, mb, mb2, msb, msb2, msa, args, max_rows, offsets ? groups : 0, s);
+  if (few) {
+    args.narrow = 1;
+    args.out_cols = 128;
+    args.n_tiles = (nout + 127) / 128;
+  }
   const int64_t bound = m_tiles * args.n_tiles;
   const int grid = (int)(bound < sm_count() ? bound : sm_count());
   if (epi == EPI_SWIGLU) return launch_tc_t<EPI_SWIGLU>(ma, mb, mb2, msb, msb2, msa, args, grid, s);

@@ -32,6 +32,7 @@ struct TcArgs {
   uint64_t wait_ns;
   int shared_group;  // group whose weights come from the second map pair (-1: none)
   int shared_a;      // 1: that group's A rows come from their own map, from row 0
+  int narrow;        // 1: 128-column tiles (one B box, N = 128), plain epilogues only
 };
 
 // ---- PTX wrappers -----------------------------------------------------------
@@ -174,11 +175,12 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* prefix, const int*
 // drains 256 accumulator columns starting at tbase's column:
 //   EPI_SWIGLU: columns c and 128 + c are the gate and up halves of hidden
 //               unit n0 + c; writes silu(gate) * up for 128 units;
-//   EPI_STORE / EPI_F32: writes the 256 columns n0 .. n0 + 255.
+//   EPI_STORE / EPI_F32: writes `ncols` (256 or 128) columns n0 .. n0 + ncols - 1.
 // Stores are masked to row_ok and to columns < nout.  All 32 lanes of the
 // warp must call it (tcgen05.ld is warp-wide).
 template <int EPI>
-__device__ __forceinline__ void epilogue_row(const TcArgs& args, uint32_t tbase, int row, bool row_ok, int n0) {
+__device__ __forceinline__ void epilogue_row(const TcArgs& args, uint32_t tbase, int row, bool row_ok, int n0,
+                                             int ncols = 256) {
   if (EPI == moe_host::EPI_SWIGLU) {
     bf16* out = reinterpret_cast<bf16*>(args.C) + (size_t)row * args.ldc;
 #pragma unroll 1
@@ -194,7 +196,7 @@ __device__ __forceinline__ void epilogue_row(const TcArgs& args, uint32_t tbase,
     }
   } else {
 #pragma unroll 1
-    for (int c = 0; c < 256; c += 32) {
+    for (int c = 0; c < ncols; c += 32) {
       uint32_t a[32];
       MOE_TMEM_LD32(tbase + c, a);
       tmem_wait_ld();
