@@ -40,7 +40,7 @@ UNIT = "tokens/s"
 # DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu
 # capture, with the sha256 of the kernel source it was taken on; reported
 # only while the source is unchanged.
-TRAFFIC = {"kernel_sha": "0be8a413ad50c125", "workload": "mixtral_bf16", "bytes": 2174398464,
+TRAFFIC = {"kernel_sha": "b067c0339cf53a9f", "workload": "mixtral_bf16", "bytes": 2173933824,
            "source": "profiles/gemm_tc_swiglu_mixtral_bf16.md"}
 
 
@@ -328,12 +328,16 @@ def run_native(args):
                     "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": traffic,
                     "peak_kind": f"HBM copy, {peaks['source']}", "algorithmic_bytes": fb["gate_up_bytes"],
                     "touched_experts": fb["touched_experts"]}
-        # library kernels per step: RMSNorm(+router), [router GEMM], top-k, 3 permute
-        # kernels, row scatter, 2 routed GEMMs, [2 shared GEMMs unless the shared
-        # expert is folded into the routed ones], combine
+        # library kernels per step: RMSNorm(+router), [router GEMM], top-k, the
+        # permute (one block-wide kernel up to 32 chunks of 256 slots whose
+        # histogram fits 96 KiB of shared memory, else three kernels), row
+        # scatter, 2 routed GEMMs, [2 shared GEMMs unless the shared expert is
+        # folded into the routed ones], combine
         router_tc = cfg.dtype == "bf16" and cfg.n_experts >= 64 and cfg.n_tokens >= 512
         shared_launches = 2 if cfg.d_ff_shared > 0 and not fb["shared_folded"] else 0
-        launches = 1 + int(router_tc) + 1 + 3 + 1 + 2 + shared_launches + 1
+        chunks = -(-cfg.n_tokens * cfg.top_k // 256)
+        permute_launches = 1 if chunks <= 32 and 4 * cfg.n_experts * (chunks + 32) <= 96 * 1024 else 3
+        launches = 1 + int(router_tc) + 1 + permute_launches + 1 + 2 + shared_launches + 1
         line = {
             "metric": METRIC, "value": round(whole_job_tokens_per_s(cfg.n_tokens, world, ms), 1), "unit": UNIT,
             "n_gpus": world,
