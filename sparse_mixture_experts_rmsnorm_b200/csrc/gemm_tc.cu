@@ -46,7 +46,8 @@ constexpr int TC_STAGES = 4;
 constexpr int TC_A_BYTES = TC_BM * TC_BK * 2;     // 16 KiB
 constexpr int TC_B_HALF_BYTES = 128 * TC_BK * 2;  // 16 KiB (one TMA box of 128 rows)
 constexpr int TC_STAGE_BYTES = TC_A_BYTES + 2 * TC_B_HALF_BYTES;
-constexpr int TC_SMEM_BYTES = TC_STAGES * TC_STAGE_BYTES + 1024;  // + alignment slack
+constexpr int TC_EPI_STAGE_BYTES = 32 * 128;  // one warp's 32 x 64 bf16 output block (TMA-store epilogue)
+constexpr int TC_SMEM_BYTES = TC_STAGES * TC_STAGE_BYTES + 4 * TC_EPI_STAGE_BYTES + 1024;  // + alignment slack
 constexpr int TC_THREADS = 192;
 
 template <int EPI>
@@ -54,7 +55,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                    const __grid_constant__ CUtensorMap map_b2, const __grid_constant__ CUtensorMap map_sb,
                    const __grid_constant__ CUtensorMap map_sb2, const __grid_constant__ CUtensorMap map_sa,
-                   const TcArgs args) {
+                   const __grid_constant__ CUtensorMap map_c, const TcArgs args) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[TC_STAGES];
   __shared__ __align__(8) uint64_t empty_bar[TC_STAGES];
@@ -229,8 +230,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       // M = 64 accumulators keep row r in lane (r / 16) * 32 + r % 16: lanes
       // 0..15 of each warp's quarter
       const bool half = tl.row_end - tl.row0 <= 64;
-      const int row = half ? tl.row0 + quarter * 16 + (lane & 15) : tl.row0 + r_local;
-      epilogue_row<EPI>(args, tbase, row, row < tl.row_end && (!half || lane < 16), tl.n0, args.narrow ? 128 : 256);
+      const int ncols = args.narrow ? 128 : 256;
+      if (EPI == moe_host::EPI_STORE && args.tma_store && !half && tl.row0 + quarter * 32 + 32 <= tl.row_end) {
+        // a whole warp of rows: 32 x 64 blocks through shared memory and TMA
+        const uint32_t stage_w = smem_base + TC_STAGES * TC_STAGE_BYTES + (uint32_t)(quarter * TC_EPI_STAGE_BYTES);
+        epilogue_warp_store_tma(&map_c, tbase, stage_w, tl.row0 + quarter * 32, tl.n0, ncols);
+      } else {
+        const int row = half ? tl.row0 + quarter * 16 + (lane & 15) : tl.row0 + r_local;
+        epilogue_row<EPI>(args, tbase, row, row < tl.row_end && (!half || lane < 16), tl.n0, ncols);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty_bar[buf]);
@@ -239,6 +247,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         bphase ^= 1u;
       }
     }
+    // the TMA stores of this warp have written global memory before the block ends
+    if (EPI == moe_host::EPI_STORE && args.tma_store && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -278,6 +288,19 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
   return fn;
 }
 
+bool make_store_map(CUtensorMap* m, void* base, int64_t rows, int cols, int ldc) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ldc * 2};
+  cuuint32_t box[2] = {64, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_tc_map(CUtensorMap* m, const void* base, int64_t rows, int k) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode();
   if (enc == nullptr) return false;
@@ -294,7 +317,7 @@ bool make_tc_map(CUtensorMap* m, const void* base, int64_t rows, int k) {
 template <int EPI>
 static moe_status launch_tc_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
                               const CUtensorMap& msb, const CUtensorMap& msb2, const CUtensorMap& msa,
-                              const moe::TcArgs& args, int grid, cudaStream_t s) {
+                              const CUtensorMap& mc, const moe::TcArgs& args, int grid, cudaStream_t s) {
   static bool attr_done[64] = {};
   int dev = current_device();
   if (dev < 64 && !attr_done[dev]) {
@@ -303,7 +326,7 @@ static moe_status launch_tc_t(const CUtensorMap& ma, const CUtensorMap& mb, cons
       return MOE_ERR_CUDA;
     attr_done[dev] = true;
   }
-  moe::gemm_tc_kernel<EPI><<<grid, moe::TC_THREADS, moe::TC_SMEM_BYTES, s>>>(ma, mb, mb2, msb, msb2, msa, args);
+  moe::gemm_tc_kernel<EPI><<<grid, moe::TC_THREADS, moe::TC_SMEM_BYTES, s>>>(ma, mb, mb2, msb, msb2, msa, mc, args);
   return launch_status();
 }
 
@@ -359,6 +382,7 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
   args.out_cols = (epi == EPI_SWIGLU) ? 128 : moe::TC_BN;
   args.n_tiles = (nout + args.out_cols - 1) / args.out_cols;
   args.narrow = 0;
+  args.tma_store = 0;
   args.C = c;
   args.ldc = ldc;
   args.hdr = hdr;
@@ -385,9 +409,19 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
   }
   const int64_t bound = m_tiles * args.n_tiles;
   const int grid = (int)(bound < sm_count() ? bound : sm_count());
-  if (epi == EPI_SWIGLU) return launch_tc_t<EPI_SWIGLU>(ma, mb, mb2, msb, msb2, msa, args, grid, s);
-  if (epi == EPI_STORE) return launch_tc_t<EPI_STORE>(ma, mb, mb2, msb, msb2, msa, args, grid, s);
-  return launch_tc_t<EPI_F32>(ma, mb, mb2, msb, msb2, msa, args, grid, s);
+  // The plain bf16 store writes whole warps' 32 x 64 blocks through TMA: one
+  // box per block instead of 16-byte pieces of 32 rows, which otherwise crowd
+  // the operand loads when K is short (measured on B200: the DeepSeek-V3-shaped
+  // down projection, K = 2048, 2.46 -> 2.32 ms; the SwiGLU epilogue writes half
+  // as much per tile and did not gain).
+  CUtensorMap mc = ma;
+  if (epi == EPI_STORE && (ldc % 8) == 0 && ((uintptr_t)c % 16) == 0) {
+    if (!make_store_map(&mc, c, max_rows, nout, ldc)) return MOE_ERR_CUDA;
+    args.tma_store = 1;
+  }
+  if (epi == EPI_SWIGLU) return launch_tc_t<EPI_SWIGLU>(ma, mb, mb2, msb, msb2, msa, mc, args, grid, s);
+  if (epi == EPI_STORE) return launch_tc_t<EPI_STORE>(ma, mb, mb2, msb, msb2, msa, mc, args, grid, s);
+  return launch_tc_t<EPI_F32>(ma, mb, mb2, msb, msb2, msa, mc, args, grid, s);
 }
 
 static int g_pairing = 0;

@@ -33,6 +33,7 @@ struct TcArgs {
   int shared_group;  // group whose weights come from the second map pair (-1: none)
   int shared_a;      // 1: that group's A rows come from their own map, from row 0
   int narrow;        // 1: 128-column tiles (one B box, N = 128), plain epilogues only
+  int tma_store;     // 1: the plain-store epilogue writes whole warps' blocks through TMA
 };
 
 // ---- PTX wrappers -----------------------------------------------------------
@@ -46,6 +47,22 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// TMA store of one box from shared memory (bulk-group completion), and the
+// bulk-group waits that guard the shared-memory buffer and the global writes.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// generic-proxy writes to shared memory become visible to the TMA (async proxy)
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -170,6 +187,45 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* prefix, const int*
   return tl;
 }
 
+// ---- plain-store epilogue of one warp's 32 rows through TMA --------------------
+// The warp's 32 rows (lane = row) of `ncols` accumulator columns go out in
+// blocks of 32 rows x 64 bf16 columns: each lane converts and writes its 128
+// bytes into `stage` (4 KiB, 1024-byte aligned) in the 128-byte-swizzled
+// layout (16-byte chunk j of row r at chunk j ^ (r % 8)), and lane 0 stores
+// the block with one TMA box at (n0 + c, row0).  Columns past the tensor are
+// clipped by the TMA.  All 32 lanes must call it.
+__device__ __forceinline__ void epilogue_warp_store_tma(const CUtensorMap* map_c, uint32_t tbase, uint32_t stage,
+                                                        int row0, int n0, int ncols) {
+  const int lane = lane_id();
+  const uint32_t my_row = stage + (uint32_t)lane * 128u;
+#pragma unroll 1
+  for (int c = 0; c < ncols; c += 64) {
+    uint32_t a[32], b[32];
+    MOE_TMEM_LD32(tbase + c, a);
+    MOE_TMEM_LD32(tbase + c + 32, b);
+    tmem_wait_ld();
+    if (lane == 0) bulk_wait_read_all();  // the previous block has left the stage
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t* v = j < 4 ? a + 8 * j : b + 8 * (j - 4);
+      const uint32_t p0 = pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1]));
+      const uint32_t p1 = pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3]));
+      const uint32_t p2 = pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5]));
+      const uint32_t p3 = pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7]));
+      const uint32_t dst = my_row + ((uint32_t)(j ^ (lane & 7)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(p0), "r"(p1), "r"(p2), "r"(p3)
+                   : "memory");
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(map_c, stage, n0 + c, row0);
+      bulk_commit();
+    }
+  }
+}
+
 // ---- epilogue of one accumulator row -----------------------------------------
 // The calling thread owns TMEM lane `tbase` (row `row` of the output) and
 // drains 256 accumulator columns starting at tbase's column:
@@ -230,6 +286,9 @@ namespace moe_host {
 // 2-D bf16 tensor map over a row-major [rows][k] matrix: box 128 rows x 64
 // columns, 128-byte swizzle, zero fill outside the matrix.
 bool make_tc_map(CUtensorMap* m, const void* base, int64_t rows, int k);
+// 2-D bf16 tensor map over the [rows][ldc] output (cols used), box 32 rows x 64
+// columns, 128-byte swizzle: the TMA-store epilogue's map.
+bool make_store_map(CUtensorMap* m, void* base, int64_t rows, int cols, int ldc);
 
 // The SM-pair kernel (gemm_tc2.cu) on maps and arguments prepared by
 // launch_gemm_tc; groups_bound = groups when offsets are given, else 0.
