@@ -209,9 +209,8 @@ def run_native(args):
     off_host = offsets.cpu().numpy()
     fb = workload_flops_bytes(cfg, off_host)
 
-    # ---- timed region: K whole steps, per-stage events on the same stream
+    # ---- timed region: K whole steps back to back, nothing recorded between them
     names = ("start", "routed", "permuted", "gate_up", "down", "shared", "combined")
-    traces = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(args.steps)]
     uuid = None
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
@@ -228,17 +227,24 @@ def run_native(args):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for i in range(args.steps):
-        step(traces[i])
+        step()
     t1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
     ms = t0.elapsed_time(t1) / args.steps
+
+    # ---- stage times: a separate pass with events recorded between the stages
+    n_traced = min(args.steps, 50)
+    traces = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(n_traced)]
+    for i in range(n_traced):
+        step(traces[i])
+    torch.cuda.synchronize()
     stage = {n: 0.0 for n in names[1:]}
     for tr in traces:
         for a, b in zip(names[:-1], names[1:]):
-            stage[b] += tr[a].elapsed_time(tr[b]) / args.steps
+            stage[b] += tr[a].elapsed_time(tr[b]) / n_traced
     st, info = moe.moe_check_device_error(ws)
     if st != 0:
         raise RuntimeError(f"device error {info}")
