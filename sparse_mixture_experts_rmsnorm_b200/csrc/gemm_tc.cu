@@ -389,6 +389,16 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
   args.wait_ns = wait_limit_ns();
   args.shared_group = (sb != nullptr && offsets) ? groups - 1 : -1;
   args.shared_a = shared_a ? 1 : 0;
+  // The plain bf16 store writes whole warps' 32 x 64 blocks through TMA: one
+  // box per block instead of 16-byte pieces of 32 rows, which otherwise crowd
+  // the operand loads when K is short (measured on B200: the DeepSeek-V3-shaped
+  // down projection, K = 2048, 2.46 -> 2.32 ms; the SwiGLU epilogue writes half
+  // as much per tile and did not gain).
+  CUtensorMap mc = ma;
+  if (epi == EPI_STORE && (ldc % 8) == 0 && ((uintptr_t)c % 16) == 0) {
+    if (!make_store_map(&mc, c, max_rows, nout, ldc)) return MOE_ERR_CUDA;
+    args.tma_store = 1;
+  }
   const int rows_per_group = max_rows / (offsets ? groups : 1);
   const int mode = tc_pairing();
   // Upper bound on the number of tiles; the exact count lives on the device.
@@ -401,7 +411,7 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
   // (down projection) by a few percent; for the SwiGLU projection the extra
   // padding of 256-row tiles outweighs the saved operand traffic.
   if (mode == 2 || (mode == 0 && rows_per_group >= 512 && epi != EPI_SWIGLU && !few))
-    return launch_gemm_tc2(epi, ma, mb, mb2, msb, msb2, msa, args, max_rows, offsets ? groups : 0, s);
+    return launch_gemm_tc2(epi, ma, mb, mb2, msb, msb2, msa, mc, args, max_rows, offsets ? groups : 0, s);
   if (few) {
     args.narrow = 1;
     args.out_cols = 128;
@@ -409,16 +419,6 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
   }
   const int64_t bound = m_tiles * args.n_tiles;
   const int grid = (int)(bound < sm_count() ? bound : sm_count());
-  // The plain bf16 store writes whole warps' 32 x 64 blocks through TMA: one
-  // box per block instead of 16-byte pieces of 32 rows, which otherwise crowd
-  // the operand loads when K is short (measured on B200: the DeepSeek-V3-shaped
-  // down projection, K = 2048, 2.46 -> 2.32 ms; the SwiGLU epilogue writes half
-  // as much per tile and did not gain).
-  CUtensorMap mc = ma;
-  if (epi == EPI_STORE && (ldc % 8) == 0 && ((uintptr_t)c % 16) == 0) {
-    if (!make_store_map(&mc, c, max_rows, nout, ldc)) return MOE_ERR_CUDA;
-    args.tma_store = 1;
-  }
   if (epi == EPI_SWIGLU) return launch_tc_t<EPI_SWIGLU>(ma, mb, mb2, msb, msb2, msa, mc, args, grid, s);
   if (epi == EPI_STORE) return launch_tc_t<EPI_STORE>(ma, mb, mb2, msb, msb2, msa, mc, args, grid, s);
   return launch_tc_t<EPI_F32>(ma, mb, mb2, msb, msb2, msa, mc, args, grid, s);

@@ -32,7 +32,8 @@ constexpr int P_STAGES = 6;
 constexpr int P_A_BYTES = 128 * TC_BK * 2;              // 16 KiB: this CTA's rows of A
 constexpr int P_B_BYTES = 128 * TC_BK * 2;              // 16 KiB: this CTA's half of B
 constexpr int P_STAGE_BYTES = P_A_BYTES + P_B_BYTES;    // 32 KiB
-constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 1024;
+constexpr int P_EPI_STAGE_BYTES = 32 * 128;  // one warp's 32 x 64 bf16 output block (TMA-store epilogue)
+constexpr int P_SMEM_BYTES = P_STAGES * P_STAGE_BYTES + 4 * P_EPI_STAGE_BYTES + 1024;
 constexpr int P_THREADS = 192;
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -99,7 +100,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                     const __grid_constant__ CUtensorMap map_b2, const __grid_constant__ CUtensorMap map_sb,
                     const __grid_constant__ CUtensorMap map_sb2, const __grid_constant__ CUtensorMap map_sa,
-                    const TcArgs args) {
+                    const __grid_constant__ CUtensorMap map_c, const TcArgs args) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[P_STAGES];   // used in the even CTA
   __shared__ __align__(8) uint64_t empty_bar[P_STAGES];
@@ -265,7 +266,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * P_BN);
       const int row = tl.row0 + r_local;
-      epilogue_row<EPI>(args, tbase, row, row < tl.row_end, tl.n0);
+      const int wrow0 = tl.row0 + (int)rank * 128 + quarter * 32;
+      if (EPI == moe_host::EPI_STORE && args.tma_store && wrow0 + 32 <= tl.row_end) {
+        // a whole warp of rows: 32 x 64 blocks through shared memory and TMA
+        const uint32_t stage_w = smem_base + P_STAGES * P_STAGE_BYTES + (uint32_t)(quarter * P_EPI_STAGE_BYTES);
+        epilogue_warp_store_tma(&map_c, tbase, stage_w, wrow0, tl.n0, 256);
+      } else {
+        epilogue_row<EPI>(args, tbase, row, row < tl.row_end, tl.n0);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(map_to_rank(&tempty_bar[buf], 0));
@@ -274,6 +282,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
         bphase ^= 1u;
       }
     }
+    // the TMA stores of this warp have written global memory before the block ends
+    if (EPI == moe_host::EPI_STORE && args.tma_store && lane == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -312,7 +322,7 @@ static int resident_pairs() {
 template <int EPI>
 static moe_status launch_tc2_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
                                const CUtensorMap& msb, const CUtensorMap& msb2, const CUtensorMap& msa,
-                               const moe::TcArgs& args, int64_t pair_bound, cudaStream_t s) {
+                               const CUtensorMap& mc, const moe::TcArgs& args, int64_t pair_bound, cudaStream_t s) {
   static bool attr_done[64] = {};
   int dev = current_device();
   if (dev < 64 && !attr_done[dev]) {
@@ -323,20 +333,21 @@ static moe_status launch_tc2_t(const CUtensorMap& ma, const CUtensorMap& mb, con
   }
   const int64_t pairs = pair_bound < resident_pairs<EPI>() ? pair_bound : resident_pairs<EPI>();
   moe::gemm_tc2_kernel<EPI><<<(unsigned)(2 * pairs), moe::P_THREADS, moe::P_SMEM_BYTES, s>>>(ma, mb, mb2, msb, msb2,
-                                                                                          msa, args);
+                                                                                          msa, mc, args);
   return launch_status();
 }
 
 // Launch of the SM-pair kernel; maps and arguments come from launch_gemm_tc.
 moe_status launch_gemm_tc2(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
                            const CUtensorMap& msb, const CUtensorMap& msb2, const CUtensorMap& msa,
-                           const moe::TcArgs& args, int64_t max_rows, int groups_bound, cudaStream_t s) {
+                           const CUtensorMap& mc, const moe::TcArgs& args, int64_t max_rows, int groups_bound,
+                           cudaStream_t s) {
   // upper bound on the pair tiles; the exact count lives on the device
   const int64_t m_pairs = (max_rows + moe::P_BM - 1) / moe::P_BM + groups_bound;
   const int64_t bound = m_pairs * args.n_tiles;
-  if (epi == EPI_SWIGLU) return launch_tc2_t<EPI_SWIGLU>(ma, mb, mb2, msb, msb2, msa, args, bound, s);
-  if (epi == EPI_STORE) return launch_tc2_t<EPI_STORE>(ma, mb, mb2, msb, msb2, msa, args, bound, s);
-  return launch_tc2_t<EPI_F32>(ma, mb, mb2, msb, msb2, msa, args, bound, s);
+  if (epi == EPI_SWIGLU) return launch_tc2_t<EPI_SWIGLU>(ma, mb, mb2, msb, msb2, msa, mc, args, bound, s);
+  if (epi == EPI_STORE) return launch_tc2_t<EPI_STORE>(ma, mb, mb2, msb, msb2, msa, mc, args, bound, s);
+  return launch_tc2_t<EPI_F32>(ma, mb, mb2, msb, msb2, msa, mc, args, bound, s);
 }
 
 }  // namespace moe_host

@@ -294,7 +294,8 @@ bool make_store_map(CUtensorMap* m, void* base, int64_t rows, int cols, int ldc)
 // launch_gemm_tc; groups_bound = groups when offsets are given, else 0.
 moe_status launch_gemm_tc2(int epi, const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
                            const CUtensorMap& msb, const CUtensorMap& msb2, const CUtensorMap& msa,
-                           const moe::TcArgs& args, int64_t max_rows, int groups_bound, cudaStream_t s);
+                           const CUtensorMap& mc, const moe::TcArgs& args, int64_t max_rows, int groups_bound,
+                           cudaStream_t s);
 
 // 0: choose per launch (SM pairs for the store / fp32 epilogues when the
 //    groups average >= 512 rows);
