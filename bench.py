@@ -209,8 +209,9 @@ def run_native(args):
     off_host = offsets.cpu().numpy()
     fb = workload_flops_bytes(cfg, off_host)
 
-    # ---- timed region: K whole steps back to back, nothing recorded between them
+    # ---- timed region: K whole steps, per-stage events on the same stream
     names = ("start", "routed", "permuted", "gate_up", "down", "shared", "combined")
+    traces = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(args.steps)]
     uuid = None
     try:
         uuid = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
@@ -227,24 +228,17 @@ def run_native(args):
     t1 = torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for i in range(args.steps):
-        step()
+        step(traces[i])
     t1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
     ms = t0.elapsed_time(t1) / args.steps
-
-    # ---- stage times: a separate pass with events recorded between the stages
-    n_traced = min(args.steps, 50)
-    traces = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(n_traced)]
-    for i in range(n_traced):
-        step(traces[i])
-    torch.cuda.synchronize()
     stage = {n: 0.0 for n in names[1:]}
     for tr in traces:
         for a, b in zip(names[:-1], names[1:]):
-            stage[b] += tr[a].elapsed_time(tr[b]) / n_traced
+            stage[b] += tr[a].elapsed_time(tr[b]) / args.steps
     st, info = moe.moe_check_device_error(ws)
     if st != 0:
         raise RuntimeError(f"device error {info}")
