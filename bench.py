@@ -40,7 +40,7 @@ UNIT = "tokens/s"
 # DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu
 # capture, with the sha256 of the kernel source it was taken on; reported
 # only while the source is unchanged.
-TRAFFIC = {"kernel_sha": "60d7a88e859e7760", "workload": "mixtral_bf16", "bytes": 2174827520,
+TRAFFIC = {"kernel_sha": "7eed3039d9afd06d", "workload": "mixtral_bf16", "bytes": 2174827520,
            "source": "profiles/gemm_tc_swiglu_mixtral_bf16.md"}
 
 
@@ -61,11 +61,16 @@ def _dist():
 
 
 def _kernel_sha():
-    """sha256 prefix of the sources of the single-SM grouped GEMM kernel."""
+    """sha256 prefix of the code of the single-SM grouped GEMM kernel: its two
+    source files with `//` comments, trailing blanks and empty lines removed, so
+    that a comment edit does not retire a traffic figure."""
     h = hashlib.sha256()
     for name in ("gemm_tc.cu", "tcgen05.cuh"):
-        with open(os.path.join(ROOT, "sparse_mixture_experts_rmsnorm_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "sparse_mixture_experts_rmsnorm_b200", "csrc", name), encoding="utf-8") as f:
+            for line in f:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

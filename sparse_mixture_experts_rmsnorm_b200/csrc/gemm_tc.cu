@@ -19,14 +19,17 @@
 //               memory) into one of two 256-column fp32 accumulators;
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (each warp owns the
 //               32 TMEM lanes = rows its rank allows), SwiGLU or plain
-//               conversion, masked stores of the rows inside the group.
+//               conversion, masked stores of the rows inside the group; the
+//               plain bf16 store sends a warp's whole 32-row blocks out
+//               through a 4 KiB shared-memory stage and a TMA store.
 // The two accumulators let the epilogue of one tile overlap the main loop
 // of the next.  A tile of at most 64 rows (a ragged expert's last tile, or
 // every tile of a decode step) runs as M = 64 MMAs; its accumulator keeps row
-// r in TMEM lane (r / 16) * 32 + r % 16, the first 16 lanes of each quarter.  For SwiGLU, B holds 128 gate rows then 128 up rows of the
-// same hidden units, so one N = 256 MMA produces both halves.  A plain-
-// epilogue launch with too few tiles to fill the SMs (the router's logits)
-// uses 128-column tiles: one B box per stage and N = 128 MMAs.
+// r in TMEM lane (r / 16) * 32 + r % 16, the first 16 lanes of each quarter.
+// For SwiGLU, B holds 128 gate rows then 128 up rows of the same hidden
+// units, so one N = 256 MMA produces both halves.  A plain-epilogue launch
+// with too few tiles to fill the SMs (the router's logits) uses 128-column
+// tiles: one B box per stage and N = 128 MMAs.
 // Tiles are numbered group-major, then n-tile, then m-tile, so CTAs working
 // at the same time share weight tiles through L2.
 // Every mbarrier wait is bounded: on time-out the block records

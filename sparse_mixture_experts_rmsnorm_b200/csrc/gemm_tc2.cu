@@ -16,8 +16,10 @@
 //   warp 1      TMEM allocation (both CTAs, cta_group::2); in the even CTA
 //               lane 0 issues the MMAs and commits to the stage and
 //               accumulator barriers of both CTAs at once (multicast commit);
-//   warps 2..5  epilogue of the CTA's own 128 rows, then one arrival per warp
-//               on the even CTA's accumulator-empty barrier.
+//   warps 2..5  epilogue of the CTA's own 128 rows (the plain bf16 store
+//               through shared memory and TMA stores, as in the single-SM
+//               kernel), then one arrival per warp on the even CTA's
+//               accumulator-empty barrier.
 // No TMA load uses cluster multicast.  Every mbarrier wait is bounded as in
 // the single-SM kernel; both CTAs always meet at the final cluster barrier.
 #include <cudaTypedefs.h>
