@@ -279,15 +279,17 @@ __global__ void selftest_wait_kernel(int32_t* hdr, uint64_t wait_ns) {
 
 namespace moe_host {
 
+// The driver's tensor-map encoder, looked up once (a function-local static, so the first calls of several host
+// threads are safe); nullptr when the driver does not export it.
 static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -321,14 +323,9 @@ template <int EPI>
 static moe_status launch_tc_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
                               const CUtensorMap& msb, const CUtensorMap& msb2, const CUtensorMap& msa,
                               const CUtensorMap& mc, const moe::TcArgs& args, int grid, cudaStream_t s) {
-  static bool attr_done[64] = {};
-  int dev = current_device();
-  if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(moe::gemm_tc_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             moe::TC_SMEM_BYTES) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    attr_done[dev] = true;
-  }
+  static SmemLimit lim;
+  const moe_status st = ensure_smem_limit(moe::gemm_tc_kernel<EPI>, moe::TC_SMEM_BYTES, lim);
+  if (st != MOE_OK) return st;
   moe::gemm_tc_kernel<EPI><<<grid, moe::TC_THREADS, moe::TC_SMEM_BYTES, s>>>(ma, mb, mb2, msb, msb2, msa, mc, args);
   return launch_status();
 }
@@ -427,9 +424,9 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
   return launch_tc_t<EPI_F32>(ma, mb, mb2, msb, msb2, msa, mc, args, grid, s);
 }
 
-static int g_pairing = 0;
-void set_tc_pairing(int mode) { g_pairing = mode; }
-int tc_pairing() { return g_pairing; }
+static std::atomic<int> g_pairing{0};
+void set_tc_pairing(int mode) { g_pairing.store(mode, std::memory_order_relaxed); }
+int tc_pairing() { return g_pairing.load(std::memory_order_relaxed); }
 
 moe_status launch_selftest_wait(int32_t* hdr, cudaStream_t s) {
   moe::selftest_wait_kernel<<<1, 32, 0, s>>>(hdr, wait_limit_ns());

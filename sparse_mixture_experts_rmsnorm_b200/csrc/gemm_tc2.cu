@@ -304,9 +304,12 @@ namespace moe_host {
 // Clusters of two that can be resident at once (one CTA per SM), per device.
 template <int EPI>
 static int resident_pairs() {
-  static int cache[64] = {};
-  int dev = current_device();
-  if (dev < 64 && cache[dev] > 0) return cache[dev];
+  static std::atomic<int> cache[64] = {};
+  const int dev = current_device();
+  if (dev >= 0 && dev < 64) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
   int n = 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(sm_count() & ~1));
@@ -317,7 +320,7 @@ static int resident_pairs() {
     n = sm_count() / 2;
   }
   if (n > sm_count() / 2) n = sm_count() / 2;
-  if (dev < 64) cache[dev] = n;
+  if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
@@ -325,14 +328,9 @@ template <int EPI>
 static moe_status launch_tc2_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
                                const CUtensorMap& msb, const CUtensorMap& msb2, const CUtensorMap& msa,
                                const CUtensorMap& mc, const moe::TcArgs& args, int64_t pair_bound, cudaStream_t s) {
-  static bool attr_done[64] = {};
-  int dev = current_device();
-  if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(moe::gemm_tc2_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             moe::P_SMEM_BYTES) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    attr_done[dev] = true;
-  }
+  static SmemLimit lim;
+  const moe_status st = ensure_smem_limit(moe::gemm_tc2_kernel<EPI>, moe::P_SMEM_BYTES, lim);
+  if (st != MOE_OK) return st;
   const int64_t pairs = pair_bound < resident_pairs<EPI>() ? pair_bound : resident_pairs<EPI>();
   moe::gemm_tc2_kernel<EPI><<<(unsigned)(2 * pairs), moe::P_THREADS, moe::P_SMEM_BYTES, s>>>(ma, mb, mb2, msb, msb2,
                                                                                           msa, mc, args);

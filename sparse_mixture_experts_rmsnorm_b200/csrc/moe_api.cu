@@ -9,8 +9,8 @@
 
 namespace moe_host {
 
-static uint64_t g_wait_ns = 2000000000ull;
-uint64_t wait_limit_ns() { return g_wait_ns; }
+static std::atomic<uint64_t> g_wait_ns{2000000000ull};
+uint64_t wait_limit_ns() { return g_wait_ns.load(std::memory_order_relaxed); }
 
 int current_device() {
   int d = 0;
@@ -19,12 +19,15 @@ int current_device() {
 }
 
 int sm_count() {
-  static int cache[64] = {};
+  static std::atomic<int> cache[64] = {};
   int d = current_device();
-  if (d < 64 && cache[d] > 0) return cache[d];
+  if (d >= 0 && d < 64) {
+    const int c = cache[d].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
   int n = 148;
   cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d);
-  if (d < 64) cache[d] = n;
+  if (d >= 0 && d < 64) cache[d].store(n, std::memory_order_relaxed);
   return n;
 }
 
@@ -377,7 +380,7 @@ moe_status moe_check_device_error(void* ws, size_t ws_bytes, void* stream, int32
 
 moe_status moe_set_wait_timeout_ns(int64_t ns) {
   if (ns < 0) return MOE_ERR_INVALID_ARG;
-  g_wait_ns = (uint64_t)ns;
+  g_wait_ns.store((uint64_t)ns, std::memory_order_relaxed);
   return MOE_OK;
 }
 

@@ -9,6 +9,9 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/moe.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
@@ -138,5 +141,26 @@ inline moe_status launch_status() {
 }
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Dynamic shared-memory limit already granted to one kernel, per device (up to 64 devices; others set it on every
+// call). The atomic keeps the common path lock-free; the mutex serialises the attribute calls, so the recorded
+// value is always one that was actually set and concurrent first calls from several host threads are safe.
+struct SmemLimit {
+  std::atomic<int> bytes[64] = {};
+  std::mutex mu;
+};
+
+// Raises `kernel`'s dynamic shared-memory limit on the current device to at least `need` bytes.
+template <typename K>
+inline moe_status ensure_smem_limit(K* kernel, int need, SmemLimit& lim) {
+  const int dev = current_device();
+  if (dev >= 0 && dev < 64 && lim.bytes[dev].load(std::memory_order_acquire) >= need) return MOE_OK;
+  std::lock_guard<std::mutex> g(lim.mu);
+  if (dev >= 0 && dev < 64 && lim.bytes[dev].load(std::memory_order_relaxed) >= need) return MOE_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, need) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (dev >= 0 && dev < 64) lim.bytes[dev].store(need, std::memory_order_release);
+  return MOE_OK;
+}
 
 }  // namespace moe_host

@@ -324,14 +324,9 @@ moe_status launch_permute(const int32_t* topk_idx, int n, int k, int e, int cap,
   // one block for small batches: histogram and running counts in shared memory
   const size_t fused_smem = sizeof(int32_t) * (size_t)e * (size_t)(nch + 32);
   if (nch <= 32 && fused_smem <= 96 * 1024) {
-    static bool attr_done[64] = {};
-    const int dev = current_device();
-    if (dev >= 64 || !attr_done[dev]) {
-      if (cudaFuncSetAttribute(moe::permute_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024) !=
-          cudaSuccess)
-        return MOE_ERR_CUDA;
-      if (dev < 64) attr_done[dev] = true;
-    }
+    static SmemLimit lim;
+    const moe_status st = ensure_smem_limit(moe::permute_fused_kernel, 96 * 1024, lim);
+    if (st != MOE_OK) return st;
     moe::permute_fused_kernel<<<1, 1024, fused_smem, s>>>(topk_idx, slots, k, e, (int)nch, cap, offsets, offsets_ext,
                                                           extra, counts, slot_row, row_token);
     return launch_status();

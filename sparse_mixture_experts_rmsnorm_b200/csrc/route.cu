@@ -278,13 +278,9 @@ static moe_status launch_rr(const void* h, const void* norm_w, const void* w_rou
   const size_t smem = sizeof(T) * (size_t)d;
   auto kern = moe::rmsnorm_router_kernel<T, V>;
   if (smem > 48 * 1024) {
-    static bool done[64] = {};
-    int dev = current_device();
-    if (dev >= 64 || !done[dev]) {
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return MOE_ERR_CUDA;
-      if (dev < 64) done[dev] = true;
-    }
+    static SmemLimit lim;
+    const moe_status st = ensure_smem_limit(kern, (int)smem, lim);
+    if (st != MOE_OK) return st;
   }
   const int epb = (logits == nullptr) ? 1 : (e <= 32 ? e : 32);
   const int yb = (logits == nullptr) ? 1 : (e + epb - 1) / epb;

@@ -395,3 +395,21 @@ def test_route_with_1024_experts_and_top_32(torch_cuda, n_tokens):
     skipped = check_routing(g, ref, cfg.top_k)
     assert set_amb.mean() < 0.05 and skipped < 0.25 * n_tokens, (set_amb.mean(), skipped)
     check_permutation(g, cfg.n_experts, -1)
+
+
+# ----------------------------------------------------------------- wide rows: the router's shared-memory limit grows
+
+def test_route_rows_wider_than_48k_of_shared_memory_in_growing_order(torch_cuda):
+    # the fused RMSNorm + router kernel keeps a row in shared memory; a later
+    # call with a wider row must raise the kernel's limit again
+    for d in (12800, 16384):  # 51,200 then 65,536 bytes of fp32 row
+        cfg = mi.LayerConfig(name="wide_rows", dtype="f32", n_tokens=8, d_model=d, n_experts=8, top_k=2, d_ff=64,
+                             seed=11)
+        g = run_gpu_layer(cfg)
+        ref = _full_oracle(cfg)
+        np.testing.assert_allclose(g["xn"], ref["xn"], rtol=2e-6, atol=1e-7)
+        check_routing(g, {"key": ref["key"], "idx": ref["idx"], "gates": ref["gates"], "scores": ref["scores"]},
+                      cfg.top_k)
+        check_permutation(g, cfg.n_experts, -1)
+        err = np.max(np.abs(g["out"] - ref["out64"]))
+        assert err <= F32_MAX_ABS, (d, err)
