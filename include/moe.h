@@ -30,6 +30,11 @@
  *    moe_check_device_error.
  *  - Calls are asynchronous: outputs are valid once the stream reaches them.
  *    Calls that share a workspace must not overlap on the GPU.
+ *  - Entry points may be called from several host threads at once.  The
+ *    library's host state is per-device caches (SM count, kernel shared-memory
+ *    limits, the tensor-map encoder) guarded by atomics and a mutex, and the
+ *    two process-wide settings (moe_set_wait_timeout_ns, moe_set_gemm_tiling),
+ *    which apply to calls that start after them.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
