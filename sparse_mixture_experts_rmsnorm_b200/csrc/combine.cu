@@ -20,6 +20,17 @@ namespace moe {
 //   out = round(acc).
 // A token whose slots are all dropped (and no shared expert) returns h exactly.
 // VEC consecutive elements per thread (VEC * sizeof(T) = 16 bytes when aligned).
+// Block (x, y) takes tokens x, x + gridDim.x, ... and the y-th of gridDim.y
+// column ranges of each row (a multiple of VEC wide), so that few tokens
+// still fill the GPU.
+__device__ __forceinline__ void column_range(int d, int vec, int& cb, int& ce) {
+  const int parts = (int)gridDim.y;
+  int w = (d + parts - 1) / parts;
+  w = (w + vec - 1) / vec * vec;
+  cb = min(d, (int)blockIdx.y * w);
+  ce = min(d, cb + w);
+}
+
 template <typename T, int VEC, int KC>
 __global__ void __launch_bounds__(128) combine_kernel(const T* __restrict__ h, const T* __restrict__ y_perm,
                                                       const int32_t* __restrict__ slot_row,
@@ -30,13 +41,15 @@ __global__ void __launch_bounds__(128) combine_kernel(const T* __restrict__ h, c
   // the folded shared expert: its rows follow the routed rows of y_perm
   if (shared_offsets != nullptr) y_shared = y_perm + (size_t)shared_offsets[E] * d;
   __shared__ float g[32];
+  int cb, ce;
+  column_range(d, VEC, cb, ce);
   for (int t = blockIdx.x; t < n; t += gridDim.x) {
     if (threadIdx.x < k) {
       rows[threadIdx.x] = slot_row[(size_t)t * k + threadIdx.x];
       g[threadIdx.x] = gates[(size_t)t * k + threadIdx.x];
     }
     __syncthreads();
-    for (int c = threadIdx.x * VEC; c < d; c += blockDim.x * VEC) {
+    for (int c = cb + threadIdx.x * VEC; c < ce; c += blockDim.x * VEC) {
       float acc[VEC];
       T tmp[VEC];
       const size_t off = (size_t)t * d + c;
@@ -105,19 +118,21 @@ __global__ void __launch_bounds__(128) combine_cols_kernel(const T* __restrict__
   if (shared_offsets != nullptr) y_shared = y_perm + (size_t)shared_offsets[E] * d;
   __shared__ float g[32];
   const int cstep = blockDim.x * VEC;
+  int cb, ce;
+  column_range(d, VEC, cb, ce);
   for (int t = blockIdx.x; t < n; t += gridDim.x) {
     if (threadIdx.x < k) {
       rows[threadIdx.x] = slot_row[(size_t)t * k + threadIdx.x];
       g[threadIdx.x] = gates[(size_t)t * k + threadIdx.x];
     }
     __syncthreads();
-    for (int c0 = threadIdx.x * VEC; c0 < d; c0 += cstep * CU) {
+    for (int c0 = cb + threadIdx.x * VEC; c0 < ce; c0 += cstep * CU) {
       float acc[CU][VEC];
       T tmp[CU][VEC];
 #pragma unroll
       for (int u = 0; u < CU; ++u) {
         const int c = c0 + u * cstep;
-        if (c >= d) break;
+        if (c >= ce) break;
         const size_t off = (size_t)t * d + c;
         if (VEC > 1) {
           *reinterpret_cast<uint4*>(tmp[u]) = *reinterpret_cast<const uint4*>(h + off);
@@ -138,7 +153,7 @@ __global__ void __launch_bounds__(128) combine_cols_kernel(const T* __restrict__
 #pragma unroll
           for (int jj = 0; jj < KC; ++jj) {
             const int j = j0 + jj;
-            if (c < d && j < k && rows[j] >= 0) {
+            if (c < ce && j < k && rows[j] >= 0) {
               const T* yr = y_perm + (size_t)rows[j] * d + c;
               if (VEC > 1) *reinterpret_cast<uint4*>(yv[u][jj]) = *reinterpret_cast<const uint4*>(yr);
               else yv[u][jj][0] = yr[0];
@@ -160,7 +175,7 @@ __global__ void __launch_bounds__(128) combine_cols_kernel(const T* __restrict__
 #pragma unroll
       for (int u = 0; u < CU; ++u) {
         const int c = c0 + u * cstep;
-        if (c >= d) break;
+        if (c >= ce) break;
         const size_t off = (size_t)t * d + c;
         if (y_shared != nullptr) {
           if (VEC > 1) {
@@ -201,7 +216,7 @@ namespace moe_host {
 template <typename T, int VEC>
 static void launch_combine_t(const void* h, const void* y_perm, const int32_t* slot_row, const float* topk_gate,
                              const void* y_shared, void* out, int n, int d, int k, const int32_t* shared_offsets,
-                             int e, int grid, cudaStream_t s) {
+                             int e, dim3 grid, cudaStream_t s) {
 #define MOE_COMBINE(KC)                                                                                    \
   moe::combine_kernel<T, VEC, KC><<<grid, 128, 0, s>>>((const T*)h, (const T*)y_perm, slot_row, topk_gate, \
                                                        (const T*)y_shared, (T*)out, n, d, k, shared_offsets, e)
@@ -222,7 +237,7 @@ moe_status launch_combine(int dtype, const void* h, const void* y_perm, const in
                           const float* topk_gate, const void* y_shared, void* out, int n, int d, int k,
                           cudaStream_t s, const int32_t* shared_offsets, int e) {
   if (n == 0) return MOE_OK;
-  int grid = n < sm_count() * 16 ? n : sm_count() * 16;
+  const dim3 grid = row_split_grid(n, d, dtype == MOE_BF16 ? 8 : 4);
   const uintptr_t addr = (uintptr_t)h | (uintptr_t)y_perm | (uintptr_t)y_shared | (uintptr_t)out;
   if (dtype == MOE_BF16) {
     if (d % 8 == 0 && addr % 16 == 0)

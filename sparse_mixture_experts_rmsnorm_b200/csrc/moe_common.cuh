@@ -142,6 +142,19 @@ inline moe_status launch_status() {
 
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Grid of the row-wise kernels (one 128-thread block per token, grid-stride):
+// up to 16 blocks per SM over the tokens and, when there are fewer tokens
+// than two blocks per SM, each row split into column ranges (at least one
+// 128-thread pass of `vec` elements each) across gridDim.y.
+inline dim3 row_split_grid(int n, int d, int vec) {
+  const int sms = sm_count();
+  const int x = n < sms * 16 ? n : sms * 16;
+  const int passes = (d + 128 * vec - 1) / (128 * vec);
+  const int want = (2 * sms + x - 1) / x;
+  const int y = passes < want ? passes : want;
+  return dim3((unsigned)x, (unsigned)(y > 1 ? y : 1));
+}
+
 // Dynamic shared-memory limit already granted to one kernel, per device (up to 64 devices; others set it on every
 // call). The atomic keeps the common path lock-free; the mutex serialises the attribute calls, so the recorded
 // value is always one that was actually set and concurrent first calls from several host threads are safe.

@@ -283,13 +283,17 @@ __global__ void __launch_bounds__(128) scatter_rows_kernel(const V* __restrict__
   __shared__ int32_t dst[33];
   const int routed = offsets[E];
   const int nd = k + (shared_rows > 0 ? 1 : 0);
+  // block (x, y): tokens x, x + gridDim.x, ..., the y-th column range of each row
+  const int w = (row_vecs + (int)gridDim.y - 1) / (int)gridDim.y;
+  const int ib = min(row_vecs, (int)blockIdx.y * w);
+  const int ie = min(row_vecs, ib + w);
   for (int t = blockIdx.x; t < n; t += gridDim.x) {
     if (threadIdx.x < k) dst[threadIdx.x] = slot_row[(size_t)t * k + threadIdx.x];
     if (threadIdx.x == 0 && shared_rows > 0) dst[k] = t < shared_rows ? routed + t : -1;
     __syncthreads();
     const V* src = xn + (size_t)t * row_vecs;
 #pragma unroll 4
-    for (int i = threadIdx.x; i < row_vecs; i += blockDim.x) {
+    for (int i = ib + threadIdx.x; i < ie; i += blockDim.x) {
       const V v = src[i];
       for (int j = 0; j < nd; ++j) {
         const int r = dst[j];
@@ -345,8 +349,10 @@ moe_status launch_gather(int dtype, const void* xn, const int32_t* slot_row, con
   if (n == 0) return MOE_OK;
   if (k > 32) return MOE_ERR_UNSUPPORTED;
   const size_t row_bytes = (size_t)d * (dtype == MOE_BF16 ? 2 : 4);
-  int grid = n < sm_count() * 16 ? n : sm_count() * 16;
   const uintptr_t addr = (uintptr_t)xn | (uintptr_t)x_perm;
+  // columns counted in 16-byte vectors, or elements for the narrower forms
+  const int vec_elems = (row_bytes % 16 == 0 && addr % 16 == 0) ? (dtype == MOE_BF16 ? 8 : 4) : 1;
+  const dim3 grid = row_split_grid(n, d, vec_elems);
   if (row_bytes % 16 == 0 && addr % 16 == 0)
     moe::scatter_rows_kernel<uint4><<<grid, 128, 0, s>>>((const uint4*)xn, slot_row, offsets, e, n, k,
                                                          (uint4*)x_perm, (int)(row_bytes / 16), shared_rows);

@@ -316,6 +316,10 @@ def test_device_wait_times_out_and_reports(torch_cuda):
          skew=(2, 8.0, 2.5)),
     # capacity 0: every routed slot dropped, the folded shared expert alone adds to h
     dict(n_tokens=64, d_model=128, n_experts=16, top_k=2, d_ff=64, d_ff_shared=64, capacity_factor=0.05),
+    # few tokens, wide rows: the row scatter and the combine split each row over
+    # 3 (top-2, two column blocks per pass) and 2 (top-6) column ranges
+    dict(n_tokens=40, d_model=2560, n_experts=8, top_k=2, d_ff=64),
+    dict(n_tokens=33, d_model=1544, n_experts=16, top_k=6, d_ff=64, d_ff_shared=64, capacity_factor=0.9),
 ])
 def test_small_bf16_layer_every_output(torch_cuda, over):
     cfg = mi.LayerConfig(name="small", dtype="bf16", seed=4, **over)
@@ -413,3 +417,15 @@ def test_route_rows_wider_than_48k_of_shared_memory_in_growing_order(torch_cuda)
         check_permutation(g, cfg.n_experts, -1)
         err = np.max(np.abs(g["out"] - ref["out64"]))
         assert err <= F32_MAX_ABS, (d, err)
+
+
+def test_fp32_layer_with_rows_split_over_blocks(torch_cuda):
+    # 20 tokens of 1028 fp32 columns: the combine splits each row into 3 column
+    # ranges (344, 344 and 340 wide); the output must not depend on the split
+    cfg = mi.LayerConfig(name="split_rows", dtype="f32", n_tokens=20, d_model=1028, n_experts=8, top_k=2, d_ff=64,
+                         seed=12)
+    g = run_gpu_layer(cfg)
+    ref = _full_oracle(cfg)
+    check_permutation(g, cfg.n_experts, -1)
+    err = np.max(np.abs(g["out"] - ref["out64"]))
+    assert err <= F32_MAX_ABS, err
