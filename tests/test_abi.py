@@ -99,6 +99,10 @@ def test_host_validation_before_any_launch():
     assert lib.moe_bias_update(0, 256, 1.0, 1e-3, 256, None) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_set_wait_timeout_ns(-1) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_check_device_error(None, 0, None, None) == moe.MOE_ERR_INVALID_ARG
+    for mode in (-1, 3, 1 << 20):
+        assert lib.moe_set_gemm_tiling(mode) == moe.MOE_ERR_INVALID_ARG
+    for mode in (1, 2, 0):  # accepted; host state only, no launch
+        assert lib.moe_set_gemm_tiling(mode) == moe.MOE_OK
 
 
 def test_python_wrapper_raises_on_error_status():
