@@ -222,7 +222,8 @@ moe_status moe_expert_ffn(const moe_config* cfg, int32_t n_groups, const int32_t
  * summed in fp32 and rounded once.  Lesson MoE block (h + sum gate * Expert);
  * glossary example (out[token] += weight * expert(token)).
  *   h [N][d], y_perm [R][d], slot_row [N*k], topk_gate [N][k] fp32,
- *   y_shared [N][d] or NULL, out [N][d] (may equal h). */
+ *   y_shared [N][d] or NULL, out [N][d] (may equal h).
+ * y_perm may be NULL only when the capacity is 0 (every slot dropped). */
 moe_status moe_combine(const moe_config* cfg, const void* h, const void* y_perm, const int32_t* slot_row,
                        const float* topk_gate, const void* y_shared, void* out, void* stream);
 

@@ -264,6 +264,8 @@ moe_status moe_combine(const moe_config* cfg, const void* h, const void* y_perm,
   if (!config_ok(cfg)) return MOE_ERR_INVALID_ARG;
   if (!config_supported(cfg)) return MOE_ERR_UNSUPPORTED;
   if (cfg->n_tokens > 0 && (!h || !slot_row || !topk_gate || !out)) return MOE_ERR_INVALID_ARG;
+  // y_perm may be NULL only when a capacity of 0 drops every slot
+  if (cfg->n_tokens > 0 && capacity_of(cfg) != 0 && !y_perm) return MOE_ERR_INVALID_ARG;
   return launch_combine(cfg->dtype, h, y_perm, slot_row, topk_gate, y_shared, out, cfg->n_tokens, cfg->d_model,
                         cfg->top_k, (cudaStream_t)stream);
 }

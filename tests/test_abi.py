@@ -97,6 +97,11 @@ def test_host_validation_before_any_launch():
     st = lib.moe_expert_ffn(ctypes.byref(good), 1, None, 100000, 256, 256, 256, 256, 128, 256, 256, 1 << 30, None)
     assert st == moe.MOE_ERR_WORKSPACE
     assert lib.moe_bias_update(0, 256, 1.0, 1e-3, 256, None) == moe.MOE_ERR_INVALID_ARG
+    # combine: the expert rows are required while any slot can be kept
+    st = lib.moe_combine(ctypes.byref(good), 256, None, 256, 256, None, 256, None)
+    assert st == moe.MOE_ERR_INVALID_ARG
+    st = lib.moe_combine(ctypes.byref(good), None, 256, 256, 256, None, 256, None)
+    assert st == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_set_wait_timeout_ns(-1) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_check_device_error(None, 0, None, None) == moe.MOE_ERR_INVALID_ARG
     for mode in (-1, 3, 1 << 20):
