@@ -285,6 +285,47 @@ def test_dropped_tokens_pass_through_on_residual():
     np.testing.assert_array_equal(res["out64"][dropped], a["h"][dropped])
 
 
+def test_partially_dropped_token_keeps_its_unrenormalised_gate():
+    # [GLOSSARY] "Load balancing and expert capacity": a slot over the limit
+    # skips its expert and the token continues on the residual for that slot.
+    # Reading: the kept slot adds gate_kept * y_kept with the gate computed
+    # over all k chosen experts (no renormalisation over the kept ones).
+    # Hand-built case, E = 3, k = 2, N = 2, C = 0.75: cap = floor(0.75*2*2/3) = 1.
+    # Token 0 chooses experts {0, 1}, token 1 chooses {0, 2}; expert 0's one
+    # place goes to token 0, so token 1 keeps only its slot on expert 2.
+    d, H = 8, 12
+    r = np.random.default_rng(5)
+    h = 0.01 * r.standard_normal((2, d))
+    h[0, 0] += 1.0
+    h[1, 1] += 1.0
+    w_router = np.zeros((3, d))
+    w_router[0, :2] = [2.0, 2.0]
+    w_router[1, :2] = [1.0, -1.0]
+    w_router[2, :2] = [-1.0, 1.0]
+    wg, wu, wd = r.standard_normal((3, H, d)) * 0.4, r.standard_normal((3, H, d)) * 0.4, r.standard_normal((3, d, H))
+    res = oracle.layer_forward(h, np.ones(d), w_router, np.zeros(3), wg, wu, wd, top_k=2, eps=1e-6, dtype="f32",
+                               capacity_factor=0.75)
+    assert res["capacity"] == 1
+    assert res["idx"].tolist() == [[0, 1], [0, 2]]
+    assert res["slot_row"].tolist() == [0, 1, -1, 2]  # token 1's slot on expert 0 is dropped
+    # the expected token-1 output, written out with torch from the definitions
+    xn = torch.nn.functional.rms_norm(torch.tensor(h), (d,), eps=float(np.float32(1e-6)))
+    p = torch.softmax(xn @ torch.tensor(w_router).T, dim=1)
+    g_kept = float(p[1, 2] / (p[1, 0] + p[1, 2]))  # gate of expert 2 over the two chosen experts
+    y2 = _torch_swiglu(xn[1:2].numpy(), wg[2], wu[2], wd[2]).numpy()[0]
+    expect = h[1] + g_kept * y2
+    np.testing.assert_allclose(res["out64"][1], expect, rtol=1e-5, atol=1e-6)
+    # the plausible wrong readings are far from it: renormalised over the kept
+    # slot (gate 1), or the kept gate scaled by 1/k
+    assert 0.01 < g_kept < 0.4 and np.linalg.norm(y2) > 0.5
+    for wrong in (h[1] + y2, h[1] + 0.5 * y2):
+        assert np.max(np.abs(res["out64"][1] - wrong)) > 0.05
+    # token 0 keeps both slots: the plain gated sum
+    g0 = (p[0, [0, 1]] / p[0, [0, 1]].sum()).numpy()
+    y0 = [_torch_swiglu(xn[0:1].numpy(), wg[e], wu[e], wd[e]).numpy()[0] for e in (0, 1)]
+    np.testing.assert_allclose(res["out64"][0], h[0] + g0[0] * y0[0] + g0[1] * y0[1], rtol=1e-5, atol=1e-6)
+
+
 # ---------------------------------------------------------------- a10 bias update
 
 def test_bias_update_exact_fp32_sign_rule():
