@@ -45,13 +45,6 @@ class LayerConfig:
     def with_(self, **kw) -> "LayerConfig":
         return replace(self, **kw)
 
-    @property
-    def capacity(self) -> int:
-        """Per-expert capacity floor(C*N*k/E), or -1 when there is no limit."""
-        if self.capacity_factor <= 0:
-            return -1
-        return int(math.floor(float(self.capacity_factor) * self.n_tokens * self.top_k / self.n_experts))
-
 
 @dataclass(frozen=True)
 class TensorSpec:

@@ -18,7 +18,6 @@ renormalised over the k chosen experts.
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 from dataclasses import dataclass
 
@@ -157,19 +156,6 @@ class Config:
     def c(self) -> MoeConfig:
         return MoeConfig(self.n_tokens, self.d_model, self.n_experts, self.top_k, self.d_ff, self.d_ff_shared,
                          MOE_BF16 if self.dtype == "bf16" else MOE_F32, self.rms_eps, self.capacity_factor)
-
-    @property
-    def capacity(self) -> int:
-        if not self.capacity_factor > 0:
-            return -1
-        c = float(ctypes.c_float(self.capacity_factor).value)
-        return int(math.floor(c * self.n_tokens * self.top_k / self.n_experts))
-
-    @property
-    def rows(self) -> int:
-        r = self.n_tokens * self.top_k
-        cap = self.capacity
-        return r if cap < 0 else min(r, self.n_experts * cap)
 
 
 def workspace_size(cfg: Config) -> int:

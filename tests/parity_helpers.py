@@ -16,6 +16,17 @@ BF16_REL_RMS = 2e-2     # bf16 layers: max |gpu - oracle| / rms(oracle)
 F32_MAX_ABS = 1e-4      # fp32 layer: max |gpu - oracle|
 
 
+def capacity(cfg) -> int:
+    """The oracle's per-expert capacity of a workload or library config (-1: none)."""
+    return oracle.capacity_limit(cfg.capacity_factor, cfg.n_tokens, cfg.top_k, cfg.n_experts)
+
+
+def expert_rows(cfg) -> int:
+    """Rows of the expert-sorted buffers: N*k, or at most E*capacity with a capacity."""
+    r, cap = cfg.n_tokens * cfg.top_k, capacity(cfg)
+    return r if cap < 0 else min(r, cfg.n_experts * cap)
+
+
 def lib_config(cfg: mi.LayerConfig):
     import sparse_mixture_experts_rmsnorm_b200 as moe
     return moe.Config(cfg.n_tokens, cfg.d_model, cfg.n_experts, cfg.top_k, cfg.d_ff, cfg.d_ff_shared,

@@ -58,7 +58,7 @@ def test_workspace_bytes_match_the_documented_regions():
     routing = N * E * 4 + 4 * N * k * 4  # logits, idx, gate, slot_row, row_token
     # bf16: xn, routing, x_perm, act, y_perm, y_shared
     c = _cfg(dtype="bf16", n_tokens=N, d_model=d, n_experts=E, top_k=k, d_ff=H, d_ff_shared=Hs)
-    R = c.rows
+    R = N * k  # no capacity: every slot keeps a row
     need = N * d * 2 + routing + 2 * R * d * 2 + max(R * H, N * Hs) * 2 + N * d * 2
     assert need <= moe.workspace_size(c) <= need + 64 * 1024
     # fp32: the same regions in 4-byte elements

@@ -1,20 +1,45 @@
 """GPU parity of the four bf16 layer workloads at their full sizes.
 
 Routing, counts, permutation and drop masks are checked on every token;
-outputs on a sample of tokens the oracle computes one by one (each sampled
-token's experts are regenerated on the host); bias updates bit-exactly.
+outputs on a stratified sample the oracle computes token by token (each
+expert's weights regenerated on the host once): the first and last kept row
+of every expert, so every expert's GEMM tiles and ragged tails are reached,
+the ends of the shared expert's group, the last rows in tile order, and some
+random tokens; bias updates bit-exactly.
 """
 import numpy as np
 import pytest
 
 import moe_inputs as mi
 import oracle
-from parity_helpers import (BF16_REL_RMS, bf16_rel_rms_err, check_permutation, check_routing, oracle_outputs,
-                            oracle_routing, rel_rms_err, run_gpu_layer, tie_masks, to_np)
+from parity_helpers import (BF16_REL_RMS, bf16_rel_rms_err, capacity, check_permutation, check_routing,
+                            oracle_outputs, oracle_routing, rel_rms_err, run_gpu_layer, tie_masks, to_np)
 
 pytestmark = pytest.mark.gpu
 
-SAMPLES = {"mixtral_bf16": 24, "dsv3_prefill_bf16": 8, "dsv3_decode_bf16": 8, "stress_bf16": 16}
+# random tokens sampled on top of the stratified ones
+SAMPLES = {"mixtral_bf16": 24, "dsv3_prefill_bf16": 32, "dsv3_decode_bf16": 64, "stress_bf16": 16}
+
+
+def stratified_tokens(offsets, row_token, eligible, n_tokens, rng, n_random, late=8):
+    """Tokens whose outputs are compared: for every expert the tokens of its
+    first and last kept rows (its ragged last tile included), the first and
+    last token (the ends of the shared expert's group, which runs last), the
+    tokens of the last `late` routed rows (late in the GEMM tile order), and
+    `n_random` more.  Only tokens marked eligible are taken; an expert whose
+    rows are all ineligible is skipped.  Returns the sorted tokens."""
+    picks = []
+    for e in range(len(offsets) - 1):
+        rows = row_token[offsets[e]:offsets[e + 1]]
+        rows = rows[eligible[rows]]
+        if rows.size:
+            picks += [rows[0], rows[-1]]
+    ends = [t for t in (0, n_tokens - 1) if n_tokens and eligible[t]]
+    tail = row_token[max(0, int(offsets[-1]) - late):int(offsets[-1])]
+    pool = np.nonzero(eligible)[0]
+    rand = rng.choice(pool, size=min(n_random, pool.size), replace=False) if pool.size else []
+    return np.unique(np.concatenate([np.asarray(picks, dtype=np.int64), np.asarray(ends, dtype=np.int64),
+                                     tail[eligible[tail]].astype(np.int64), np.asarray(rand, dtype=np.int64)]))
 
 
 @pytest.mark.parametrize("name", list(SAMPLES))
@@ -29,26 +54,31 @@ def test_config_parity(name):
     np.testing.assert_array_equal(g["xn"], ref["xn"])
     skipped = check_routing(g, ref, k)
     assert skipped <= max(2, 0.01 * N), skipped
-    cap = cfg.capacity
+    cap = capacity(cfg)
     check_permutation(g, E, cap)
 
     # drop decisions against the oracle's own routing: equal up to the first
     # token whose routing was ambiguous (a near tie) when a capacity applies
-    _, ref_slot, _ = oracle.permute(ref["idx"], E, cap)
+    ref_off, ref_slot, ref_rt = oracle.permute(ref["idx"], E, cap)
     ref_keep = (ref_slot >= 0).reshape(N, k)
     gpu_keep = (g["slot_row"] >= 0).reshape(N, k)
     _, order_amb = tie_masks(ref["key"], k)
     upto = N if cap < 0 or not order_amb.any() else int(np.argmax(order_amb))
     assert np.array_equal(gpu_keep[:upto], ref_keep[:upto])
 
-    # sampled outputs
+    # sampled outputs: a row of every expert, chosen from the oracle's own
+    # permutation among the tokens whose routing is unambiguous
     rng = np.random.default_rng(0)
-    ok_tokens = np.nonzero(~order_amb[:upto])[0]
-    tokens = np.unique(rng.choice(ok_tokens, size=min(SAMPLES[name], ok_tokens.size), replace=False))
-    dropped_any = np.nonzero(~ref_keep[:upto].all(axis=1) & ~order_amb[:upto])[0]
+    eligible = ~order_amb
+    eligible[upto:] = False
+    tokens = stratified_tokens(ref_off, ref_rt, eligible, N, rng, SAMPLES[name])
+    dropped_any = np.nonzero(~ref_keep[:upto].all(axis=1) & eligible[:upto])[0]
     if dropped_any.size:
         tokens = np.unique(np.concatenate([tokens, rng.choice(dropped_any, size=min(8, dropped_any.size),
                                                               replace=False)]))
+    covered = np.unique(ref["idx"][tokens][ref_keep[tokens]])
+    reachable = np.unique(ref["idx"][eligible][ref_keep[eligible]])
+    assert np.array_equal(covered, reachable), (covered.size, reachable.size)
     ref_out = oracle_outputs(cfg, ref, tokens, ref["idx"], ref["gates"], ref_keep)
     got = g["out"][tokens]
     # the tolerance bounds the arithmetic; storing out in bf16 adds up to half
@@ -56,8 +86,9 @@ def test_config_parity(name):
     err = bf16_rel_rms_err(got, ref_out)
     raw = rel_rms_err(got, ref_out)
     raw_delta = rel_rms_err(got - ref["h"][tokens], ref_out - ref["h"][tokens])
-    print(f"{name}: beyond-storage max err/rms(out) = {err:.3e}; raw max|err|/rms(out) = {raw:.3e}, "
-          f"on out-h = {raw_delta:.3e}; tokens {tokens.size}, skipped ties {skipped}, "
+    print(f"PARITY {name}: beyond-storage max err/rms(out) = {err:.3e}; raw max|err|/rms(out) = {raw:.3e}; "
+          f"raw max|err| on out-h / rms(out-h) = {raw_delta:.3e}; tokens {tokens.size}, experts covered "
+          f"{covered.size} of {E}{' + shared' if cfg.d_ff_shared else ''}, skipped ties {skipped}, "
           f"dropped slots {int((~gpu_keep).sum())}")
     assert err <= BF16_REL_RMS, err
 

@@ -14,8 +14,8 @@ import pytest
 
 import moe_inputs as mi
 import oracle
-from parity_helpers import (BF16_REL_RMS, F32_MAX_ABS, bf16_rel_rms_err, check_permutation, check_routing,
-                            lib_config, oracle_routing, rel_rms_err, run_gpu_layer, tie_masks, to_np)
+from parity_helpers import (BF16_REL_RMS, F32_MAX_ABS, bf16_rel_rms_err, capacity, check_permutation,
+                            check_routing, lib_config, oracle_routing, rel_rms_err, run_gpu_layer, tie_masks, to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -104,7 +104,7 @@ def test_tiny_fp32_layer_with_shared_expert_and_capacity(torch_cuda):
     ref = _full_oracle(cfg)
     check_routing(g, {"key": ref["key"], "idx": ref["idx"], "gates": ref["gates"], "scores": ref["scores"]},
                   cfg.top_k)
-    check_permutation(g, cfg.n_experts, cfg.capacity)
+    check_permutation(g, cfg.n_experts, capacity(cfg))
     assert (g["slot_row"] < 0).any()
     err = np.max(np.abs(g["out"] - ref["out64"]))
     assert err <= F32_MAX_ABS, err
@@ -166,7 +166,7 @@ def test_glossary_example_permutation(torch_cuda, capacity_factor, expect_offset
     torch.cuda.synchronize()
     off = offsets.cpu().tolist()
     assert off == expect_offsets
-    cap = lc.capacity
+    cap = capacity(lc)
     ref_off, ref_slot, ref_rt = oracle.permute(np.array(fx["experts_per_token"]), E, cap)
     assert off == ref_off.tolist()
     assert slot_row.cpu().tolist() == ref_slot.tolist()
@@ -328,7 +328,7 @@ def test_small_bf16_layer_every_output(torch_cuda, over):
     np.testing.assert_array_equal(g["xn"], ref["xn"])
     check_routing(g, {"key": ref["key"], "idx": ref["idx"], "gates": ref["gates"], "scores": ref["scores"]},
                   cfg.top_k)
-    check_permutation(g, cfg.n_experts, cfg.capacity)
+    check_permutation(g, cfg.n_experts, capacity(cfg))
     err = bf16_rel_rms_err(g["out"], ref["out64"])
     print(f"small bf16 layer {over}: beyond-storage max err/rms {err:.3e}")
     assert err <= BF16_REL_RMS, err
