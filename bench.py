@@ -6,8 +6,11 @@ A step is one whole forward pass of the layer (RMSNorm, router, top-k,
 counting-sort permute and gather, grouped SwiGLU experts on the tensor
 cores, shared expert, gated combine + residual) over one batch of N tokens
 of seeded synthetic data, inputs and weights resident in HBM.  The default
-workload is the Mixtral-8x7B-shaped layer (N = 4096 tokens, d_model 4096,
-8 experts, top-2, SwiGLU hidden 14336, bf16 storage, fp32 accumulation).
+workload is the largest one that fits one GPU, the DeepSeek-V3-shaped
+prefill layer (N = 8192 tokens, d_model 7168, 256 routed experts, top-8,
+SwiGLU hidden 2048, one always-on shared expert of hidden 2048, bf16
+storage, fp32 accumulation); --workload names the others (mixtral_bf16,
+dsv3_decode_bf16, stress_bf16, tiny_fp32).
 
 Under torchrun every rank runs an independent replica of the layer on its
 own GPU (the layer shards by tokens and needs no exchange); the time is the
@@ -23,6 +26,7 @@ row counts, one JSON line; it is context for the roofline, not the bench line.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import math
@@ -75,24 +79,35 @@ def _kernel_sha():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """nvidia-smi clock / power / throttle-reason samples every 20 ms; the
+    summary keeps the samples whose timestamps fall inside the timed region
+    (begin() .. end())."""
 
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    PERIOD_MS = 20
 
     def __init__(self, uuid: str | None):
         self.proc = None
         self.uuid = uuid
+        self.t_begin = self.t_end = None
 
     def start(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", str(self.PERIOD_MS)]
         if self.uuid:
             cmd += ["-i", self.uuid]
         try:
             self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+
+    def begin(self):
+        self.t_begin = datetime.datetime.now()
+
+    def end(self):
+        self.t_end = datetime.datetime.now()
 
     def stop(self):
         if self.proc is None:
@@ -106,20 +121,27 @@ class ClockSampler:
         rows = []
         for line in out.strip().splitlines():
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) != 7:
+            if len(parts) != 8:
                 continue
             try:
-                rows.append((float(parts[0]), float(parts[1]), float(parts[2]), parts[3:]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+                rows.append((ts, float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
             except ValueError:
                 continue
         if not rows:
             return None
+        inside = [r for r in rows if self.t_begin is not None and self.t_end is not None
+                  and self.t_begin <= r[0] <= self.t_end]
+        window = "timed region"
+        if not inside:  # a region shorter than one sampling period: the samples around it
+            inside, window = rows, "whole run (no sample fell inside the timed region)"
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v.lower() == "active"})
-        loaded = [r[0] for r in rows if r[2] > 300.0] or [r[0] for r in rows]
-        loaded.sort()
-        return {"sm_mhz": loaded[len(loaded) // 2], "sm_max_mhz": rows[0][1], "reasons": reasons,
-                "samples": len(rows), "power_w_max": max(r[2] for r in rows)}
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[4]) if v.lower() == "active"})
+        mhz = sorted(r[1] for r in inside)
+        return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": inside[0][2], "reasons": reasons,
+                "samples": len(inside), "period_ms": self.PERIOD_MS, "window": window,
+                "sm_mhz_min": mhz[0], "sm_mhz_max": mhz[-1], "power_w_max": max(r[3] for r in inside),
+                "power_w_median": sorted(r[3] for r in inside)[len(inside) // 2]}
 
 
 def workload_flops_bytes(cfg, offsets_host=None):
@@ -158,6 +180,19 @@ def workload(args):
         cur = getattr(cfg, k)
         over[k] = type(cur)(v) if not isinstance(cur, bool) else v.lower() in ("1", "true")
     return cfg.with_(**over) if over else cfg
+
+
+def preroll_steps(step, seconds: float) -> int:
+    """Run steps back to back for about `seconds` of wall time (synchronising
+    every few steps to read the clock); returns how many ran."""
+    import torch
+    n, t_end = 0, time.perf_counter() + seconds
+    while time.perf_counter() < t_end:
+        for _ in range(4):
+            step()
+        n += 4
+        torch.cuda.synchronize()
+    return n
 
 
 def max_over_ranks(values, device):
@@ -225,17 +260,28 @@ def run_native(args):
     sampler = ClockSampler(uuid) if rank == 0 else None
     if sampler:
         sampler.start()
-        time.sleep(0.3)
+    # untimed pre-roll of about PREROLL_S seconds of back-to-back steps, so the
+    # timed steps run at the clock the GPU settles at under this load (the
+    # 1 kW power cap lowers it within a second or two); every rank runs the
+    # same number of pre-roll steps
+    pre = preroll_steps(step, args.preroll)
+    pre = int(max_over_ranks([pre], "cuda")[0]) - pre
+    for _ in range(pre):
+        step()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    if sampler:
+        sampler.begin()
     t0.record(stream)
     for i in range(args.steps):
         step(traces[i])
     t1.record(stream)
     torch.cuda.synchronize()
+    if sampler:
+        sampler.end()
     if world > 1:
         dist.barrier()
     clocks = sampler.stop() if sampler else None
@@ -309,30 +355,34 @@ def run_native(args):
         gu_tflops = fb["gate_up_flops"] / (gu_ms * 1e-3) / 1e12
         expert_ms = stage["gate_up"] + stage["down"] + stage["shared"]
         expert_tflops = fb["expert_flops"] / (expert_ms * 1e-3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
+        # The timed region is a burst of K steps after a short pre-roll, so the
+        # fraction is taken of the burst peak; the power-capped sustained peak
+        # is reported beside it.
+        peak, peak_sus = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
         sha = _kernel_sha()
         traffic = TRAFFIC.get("bytes") if TRAFFIC.get("kernel_sha") == sha and \
-            TRAFFIC.get("workload") == args.workload else None
+            TRAFFIC.get("workload") == args.workload and not args.set else None
+        kernel = ("grouped gate/up + SwiGLU GEMM (tcgen05)" +
+                  (" incl. the folded shared expert" if fb["shared_folded"] else ""))
         # the dominant kernel is bound by whichever of its FLOPs and its bytes
         # takes longer at the measured peaks
         t_tensor = fb["gate_up_flops"] / (peak * 1e12)
         t_hbm = fb["gate_up_bytes"] / (peaks["hbm_gbs"] * 1e9)
         if t_tensor >= t_hbm:
-            roof = {"kernel": "grouped gate/up + SwiGLU GEMM (tcgen05)" +
-                              (" incl. the folded shared expert" if fb["shared_folded"] else ""), "bound": "tensor",
-                    "achieved": round(gu_tflops, 1), "peak": peak, "unit": "TFLOP/s",
-                    "frac": round(gu_tflops / peak, 4), "traffic": traffic,
-                    "peak_kind": f"bf16 dense, sustained, {peaks['source']}",
-                    "frac_of_burst": round(gu_tflops / peaks["bf16_tflops"], 4),
-                    "algorithmic_flops": fb["gate_up_flops"]}
+            roof = {"kernel": kernel, "bound": "tensor", "achieved": round(gu_tflops, 1), "peak": peak,
+                    "unit": "TFLOP/s", "frac": round(gu_tflops / peak, 4), "traffic": traffic,
+                    "peak_kind": f"bf16 dense, burst, {peaks['source']}",
+                    "frac_of_sustained": round(gu_tflops / peak_sus, 4), "peak_sustained": peak_sus,
+                    "algorithmic_flops": fb["gate_up_flops"], "algorithmic_bytes": fb["gate_up_bytes"],
+                    "hbm_gbs_achieved": round(fb["gate_up_bytes"] / (gu_ms * 1e-3) / 1e9, 1)}
         else:
             gbs = fb["gate_up_bytes"] / (gu_ms * 1e-3) / 1e9
-            roof = {"kernel": "grouped gate/up + SwiGLU GEMM (tcgen05)" +
-                              (" incl. the folded shared expert" if fb["shared_folded"] else ""), "bound": "hbm",
-                    "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": traffic,
+            roof = {"kernel": kernel, "bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": traffic,
                     "peak_kind": f"HBM copy, {peaks['source']}", "algorithmic_bytes": fb["gate_up_bytes"],
                     "touched_experts": fb["touched_experts"]}
+        roof["traffic_source"] = TRAFFIC.get("source") if traffic is not None else None
+        roof["ms"] = round(gu_ms, 4)
         # library kernels per step: RMSNorm(+router), [router GEMM], top-k, the
         # permute (one block-wide kernel up to 32 chunks of 256 slots whose
         # histogram fits 96 KiB of shared memory, else three kernels), row
@@ -356,8 +406,9 @@ def run_native(args):
                        "parallelism": f"replicas x{world} (token-sharded, no exchange)",
                        "l2": "inputs larger than L2 (expert weights stream from HBM every step)"},
             "roofline": roof,
-            "expert_gemm": {"tflops": round(expert_tflops, 1), "frac_sustained": round(expert_tflops / peak, 4),
-                            "ms": round(expert_ms, 4)},
+            "expert_gemm": {"tflops": round(expert_tflops, 1), "frac_burst": round(expert_tflops / peak, 4),
+                            "frac_sustained": round(expert_tflops / peak_sus, 4), "ms": round(expert_ms, 4),
+                            "flops": fb["expert_flops"], "kept_rows": fb["rows"]},
             "stage_ms": {n: round(v, 4) for n, v in stage.items()},
             "e2e": {"value": round(whole_job_tokens_per_s(cfg.n_tokens, world, e2e_ms), 1), "unit": UNIT,
                     "pipelining": "double-buffered: input copy, layer and output copy on three streams",
@@ -366,8 +417,7 @@ def run_native(args):
             "gpu_launches": launches * args.steps,
             "clocks": clocks,
         }
-        weight_bytes = 8 * 3 * (cfg.n_experts * cfg.d_ff + cfg.d_ff_shared) * cfg.d_model
-        if world == 1 and not args.no_cpu_baseline and weight_bytes < 24e9:
+        if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(cfg)
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -385,13 +435,60 @@ def _cores():
     return os.cpu_count()
 
 
-def _oracle_sample(cfg, n_tok: int):
-    """The sample's inputs: the first n_tok tokens of the workload and the full weights (host)."""
-    import moe_inputs as mi
-    import numpy as np
-    sub = cfg.with_(n_tokens=n_tok)
-    a = {n: mi.host_tensor(sub, n).astype(np.float64) for n in mi.layer_tensor_specs(sub)}
-    return sub, a
+# Host memory the oracle sample may hold as float64 expert weights.
+ORACLE_WEIGHT_BUDGET = 12e9
+
+
+class _OracleSample:
+    """Host inputs of a bounded oracle sample of a workload: its first n
+    tokens, the router, and the weights of only those experts the n tokens
+    route to (plus the shared expert), widened to float64 outside the timed
+    region.  The oracle reads the stacked expert weights only at experts with
+    kept slots, so a dict keyed by expert index stands in for them.  Expert
+    weights are regenerated from the seeded generator once and kept across
+    samples of the same workload."""
+
+    def __init__(self, cfg):
+        self.cfg = cfg
+        self.experts = {}
+        self.shared = None
+        self.bytes_per_expert = 8.0 * 3 * cfg.d_ff * cfg.d_model
+
+    def max_tokens(self) -> int:
+        """Most tokens whose touched experts fit ORACLE_WEIGHT_BUDGET (at most k new experts a token)."""
+        c = self.cfg
+        if c.n_experts * self.bytes_per_expert <= ORACLE_WEIGHT_BUDGET:
+            return c.n_tokens
+        return int(max(1, min(c.n_tokens, ORACLE_WEIGHT_BUDGET // (self.bytes_per_expert * c.top_k))))
+
+    def inputs(self, n_tok: int):
+        import numpy as np
+
+        import moe_inputs as mi
+        import oracle
+        sub = self.cfg.with_(n_tokens=n_tok)
+        a = {n: mi.host_tensor(sub, n).astype(np.float64) for n in ("h", "norm_w", "w_router", "bias")}
+        # the experts these tokens route to (the oracle's own routing, before any capacity cut)
+        xn = oracle.rmsnorm(a["h"], a["norm_w"], sub.rms_eps, sub.dtype)
+        _, scores = oracle.router_scores(xn, a["w_router"])
+        idx, _ = oracle.select_topk(scores, a["bias"], sub.top_k)
+        touched = sorted(set(np.unique(idx).tolist()))
+        for e in touched:
+            if e not in self.experts:
+                sl = slice(e, e + 1)
+                self.experts[e] = tuple(mi.host_tensor(sub, n, rows=sl)[0].astype(np.float64)
+                                        for n in ("w_gate", "w_up", "w_down"))
+        for e in list(self.experts):
+            if e not in touched:
+                del self.experts[e]
+        a["w_gate"] = {e: w[0] for e, w in self.experts.items()}
+        a["w_up"] = {e: w[1] for e, w in self.experts.items()}
+        a["w_down"] = {e: w[2] for e, w in self.experts.items()}
+        if sub.d_ff_shared > 0:
+            if self.shared is None:
+                self.shared = {n: mi.host_tensor(sub, n).astype(np.float64) for n in ("ws_gate", "ws_up", "ws_down")}
+            a.update(self.shared)
+        return sub, a, len(touched)
 
 
 def _oracle_step(sub, a):
@@ -402,21 +499,34 @@ def _oracle_step(sub, a):
                                 ws_up=a.get("ws_up"), ws_down=a.get("ws_down"))
 
 
-def _calibrated_tokens(cfg, seconds: float) -> int:
-    """Tokens of a sample that keeps the oracle busy for about `seconds`."""
-    probe = 32
-    sub, a = _oracle_sample(cfg, probe)
+def _calibrated_sample(cfg, seconds: float):
+    """A sample whose oracle pass takes about `seconds` (within the weight budget):
+    returns (sample, sub, inputs, touched experts)."""
+    smp = _OracleSample(cfg)
+    n_max = smp.max_tokens()
+    probe = min(32, n_max)
+    sub, a, touched = smp.inputs(probe)
     t0 = time.perf_counter()
     _oracle_step(sub, a)
     dt = max(time.perf_counter() - t0, 1e-3)
-    return int(max(8, min(cfg.n_tokens, probe * seconds / dt)))
+    n = int(max(1, min(n_max, probe * seconds / dt)))
+    if n != probe:
+        sub, a, touched = smp.inputs(n)
+    return smp, sub, a, touched
+
+
+def _sample_note(cfg, sub, touched):
+    return (f"the first {sub.n_tokens} of the {cfg.n_tokens} tokens of the {cfg.name} workload through the "
+            f"float64 numpy oracle (routing, {touched} touched routed experts"
+            f"{' + the shared expert' if cfg.d_ff_shared else ''}, combine); their weights regenerated from the "
+            f"seeded generator and resident on the host as float64 before timing")
 
 
 def cpu_baseline(cfg, seconds: float = 12.0, cap: float = 30.0):
     """The oracle on a bounded sample: the first n tokens of the workload,
     passed through repeatedly until about `seconds` of host time (at most `cap`)."""
-    n_tok = _calibrated_tokens(cfg, seconds)
-    sub, a = _oracle_sample(cfg, n_tok)
+    _, sub, a, touched = _calibrated_sample(cfg, seconds)
+    n_tok = sub.n_tokens
     done, dt, passes = 0, 0.0, 0
     t0 = time.perf_counter()
     while dt < seconds and (passes == 0 or dt * (passes + 1) / passes < cap):
@@ -425,8 +535,7 @@ def cpu_baseline(cfg, seconds: float = 12.0, cap: float = 30.0):
         done += n_tok
         dt = time.perf_counter() - t0
     return {"value": round(done / dt, 3), "unit": UNIT, "cores": _cores(), "kind": "oracle",
-            "sample": f"{passes} pass(es) of the first {n_tok} of the {cfg.n_tokens} tokens of the {cfg.name} "
-                      f"workload through the float64 numpy oracle, weights resident on the host ({dt:.1f} s)"}
+            "sample": f"{passes} pass(es) of {_sample_note(cfg, sub, touched)} ({dt:.1f} s timed)"}
 
 
 def run_reference(args):
@@ -435,8 +544,7 @@ def run_reference(args):
         return
     cfg = workload(args)
     # each step a bounded sample: the whole run stays near two minutes
-    n_tok = _calibrated_tokens(cfg, 120.0 / (args.steps + args.warmup))
-    sub, a = _oracle_sample(cfg, n_tok)
+    _, sub, a, touched = _calibrated_sample(cfg, 120.0 / (args.steps + args.warmup))
     for _ in range(args.warmup):
         _oracle_step(sub, a)
     t0 = time.perf_counter()
@@ -451,8 +559,7 @@ def run_reference(args):
         "config": {"workload": args.workload, "n_tokens": cfg.n_tokens, "d_model": cfg.d_model,
                    "n_experts": cfg.n_experts, "top_k": cfg.top_k, "d_ff": cfg.d_ff},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": _cores(), "kind": "oracle",
-                         "sample": f"each step: the first {sub.n_tokens} tokens of {cfg.name} through the "
-                                   f"float64 numpy oracle on the host cores"},
+                         "sample": f"each step: {_sample_note(cfg, sub, touched)}"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
@@ -550,7 +657,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="mixtral_bf16")
+    ap.add_argument("--workload", default="dsv3_prefill_bf16")
+    ap.add_argument("--preroll", type=float, default=2.0,
+                    help="seconds of untimed back-to-back steps before the timed region")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--library-baseline", action="store_true",
