@@ -194,8 +194,10 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const voi
  *  - E * ceil(N*k / 256) must not exceed MOE_NOALLOC_HIST_INTS, else the
  *    call returns MOE_ERR_WORKSPACE and enqueues nothing;
  *  - the first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) and caches it; make that first call before any
- *    stream capture;
+ *    (cudaGetSymbolAddress) and caches it for the process; make that first
+ *    call before any stream capture.  The cached address belongs to the
+ *    device's primary context: after cudaDeviceReset, or with another
+ *    driver-API context current, the call is not supported;
  *  - every call on a device shares the one array: calls that overlap on the
  *    GPU (other streams, other threads) race and give wrong results.
  * The call allocates nothing and frees nothing. */

@@ -42,9 +42,14 @@ struct Layout {
   int64_t act_elems; // max(R * H, N * Hs)
 };
 
+// floor(C*N*k/E), clamped to N*k: an expert never receives more than N*k
+// slots, so any larger cap keeps every slot, and the clamped value always fits
+// an int (config_ok bounds N*k).
 int64_t capacity_of(const moe_config* c) {
   if (!(c->capacity_factor > 0.f)) return -1;
-  return (int64_t)floor((double)c->capacity_factor * (double)c->n_tokens * (double)c->top_k / (double)c->n_experts);
+  const int64_t slots = (int64_t)c->n_tokens * c->top_k;
+  const double cap = floor((double)c->capacity_factor * (double)c->n_tokens * (double)c->top_k / (double)c->n_experts);
+  return cap >= (double)slots ? slots : (int64_t)cap;
 }
 
 static Layout layout_of(const moe_config* c) {

@@ -37,14 +37,26 @@ std::mutex g_setup_mutex;
 int32_t* g_hist_ptr[kMaxDevices] = {};
 
 // Device address of g_perm_hist for the current device (set-up on first use).
+// The address is cached per device ordinal for the life of the process: it
+// belongs to the device's primary context, the one the runtime API uses.  A
+// cudaDeviceReset, or a caller that makes another driver-API context
+// current, would need the lookup again; neither is supported by this call.
+// A failed lookup clears the runtime's error state, so the failure is
+// reported once, by this call, and not again by the next launch check.
 moe_status hist_address(int32_t** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
   if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_setup_mutex);
   if (g_hist_ptr[dev] == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_perm_hist) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+    if (cudaGetSymbolAddress(&p, g_perm_hist) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
     g_hist_ptr[dev] = static_cast<int32_t*>(p);
   }
   *out = g_hist_ptr[dev];
