@@ -220,8 +220,9 @@ def run_native(args):
     world, rank, local = _dist()
     torch.cuda.set_device(local)
     if world > 1:
-        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     cfg = workload(args)
+    moe.moe_set_gemm_tiling(args.tiling)
     lc = moe.Config(cfg.n_tokens, cfg.d_model, cfg.n_experts, cfg.top_k, cfg.d_ff, cfg.d_ff_shared, cfg.dtype,
                     cfg.rms_eps, cfg.capacity_factor)
     # each replica gets its own tokens (seed = rank), the same weights (seed 0)
@@ -404,6 +405,7 @@ def run_native(args):
                        "n_experts": cfg.n_experts, "top_k": cfg.top_k, "d_ff": cfg.d_ff,
                        "d_ff_shared": cfg.d_ff_shared, "capacity_factor": cfg.capacity_factor,
                        "parallelism": f"replicas x{world} (token-sharded, no exchange)",
+                       "gemm_tiling": args.tiling, "preroll_s": args.preroll,
                        "l2": "inputs larger than L2 (expert weights stream from HBM every step)"},
             "roofline": roof,
             "expert_gemm": {"tflops": round(expert_tflops, 1), "frac_burst": round(expert_tflops / peak, 4),
@@ -658,6 +660,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="dsv3_prefill_bf16")
+    ap.add_argument("--tiling", type=int, default=0,
+                    help="moe_set_gemm_tiling mode of the expert GEMMs (0 = automatic, the library's default)")
     ap.add_argument("--preroll", type=float, default=2.0,
                     help="seconds of untimed back-to-back steps before the timed region")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])

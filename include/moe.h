@@ -262,9 +262,12 @@ moe_status moe_set_wait_timeout_ns(int64_t ns);
 /* Tile shape of the bf16 grouped expert GEMMs for launches after this call
  * (process-wide): 0 = choose per launch (the default: SM-pair 256-row tiles
  * for the down projection and the router when the groups average at least
- * 512 rows, single-SM 128-row tiles otherwise),
- * 1 = single-SM tiles, 2 = SM-pair tiles.  Results are the same up to
- * floating-point summation order; this is a performance control. */
+ * 512 rows, single-SM 128-row tiles otherwise), 1 = single-SM tiles,
+ * 2 = SM-pair tiles, 3 = SM-pair tiles with the operands swapped for the
+ * expert GEMMs: 256 weight rows on M, up to 256 of a group's rows on N,
+ * padded to 16 (the router keeps the automatic choice).  Results are
+ * the same up to floating-point summation order; this is a performance
+ * control.  MOE_ERR_INVALID_ARG for any other mode. */
 moe_status moe_set_gemm_tiling(int32_t mode);
 
 /* Launch one block that waits on a workspace flag that nothing sets, with

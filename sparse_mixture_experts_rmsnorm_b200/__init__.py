@@ -263,7 +263,8 @@ def moe_set_wait_timeout_ns(ns: int):
 
 
 def moe_set_gemm_tiling(mode: int):
-    """0 = automatic, 1 = single-SM 128-row tiles, 2 = SM-pair 256-row tiles."""
+    """0 = automatic, 1 = single-SM 128-row tiles, 2 = SM-pair 256-row tiles,
+    3 = operands swapped on SM pairs (weight rows on M, each group's rows on N)."""
     _check(_lib.moe_set_gemm_tiling(int(mode)), "moe_set_gemm_tiling")
 
 

@@ -306,12 +306,14 @@ bool make_store_map(CUtensorMap* m, void* base, int64_t rows, int cols, int ldc)
   return r == CUDA_SUCCESS;
 }
 
-bool make_tc_map(CUtensorMap* m, const void* base, int64_t rows, int k) {
+bool make_tc_map(CUtensorMap* m, const void* base, int64_t rows, int k) { return make_tc_map_rows(m, base, rows, k, 128); }
+
+bool make_tc_map_rows(CUtensorMap* m, const void* base, int64_t rows, int k, int box_rows) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)k * 2};
-  cuuint32_t box[2] = {(cuuint32_t)moe::TC_BK, 128};
+  cuuint32_t box[2] = {(cuuint32_t)moe::TC_BK, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -400,7 +402,13 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
     args.tma_store = 1;
   }
   const int rows_per_group = max_rows / (offsets ? groups : 1);
-  const int mode = tc_pairing();
+  const int forced = tc_pairing();
+  // Operands swapped on SM pairs (gemm_swap.cu): weight rows on M, the
+  // group's rows on N in chunks of at most 256 padded to 16.  Measured slower
+  // than the tilings below on every workload so far, so only on request.
+  if (epi != EPI_F32 && forced == 3)
+    return launch_gemm_swap(epi, a, b, b2, offsets, groups, max_rows, nout, k, c, ldc, hdr, s, sb, sb2, sa, sa_rows);
+  const int mode = forced == 3 ? 0 : forced;  // the router's fp32 logits: the automatic choice
   // Upper bound on the number of tiles; the exact count lives on the device.
   const int64_t m_tiles = (int64_t)(max_rows + moe::TC_BM - 1) / moe::TC_BM + (offsets ? groups : 0);
   // A plain-epilogue launch that would leave more than half the SMs idle

@@ -392,7 +392,7 @@ moe_status moe_set_wait_timeout_ns(int64_t ns) {
 }
 
 moe_status moe_set_gemm_tiling(int32_t mode) {
-  if (mode < 0 || mode > 2) return MOE_ERR_INVALID_ARG;
+  if (mode < 0 || mode > 3) return MOE_ERR_INVALID_ARG;
   set_tc_pairing(mode);
   return MOE_OK;
 }

@@ -286,6 +286,8 @@ namespace moe_host {
 // 2-D bf16 tensor map over a row-major [rows][k] matrix: box 128 rows x 64
 // columns, 128-byte swizzle, zero fill outside the matrix.
 bool make_tc_map(CUtensorMap* m, const void* base, int64_t rows, int k);
+// The same with a box of `box_rows` rows (8 .. 256) x 64 columns.
+bool make_tc_map_rows(CUtensorMap* m, const void* base, int64_t rows, int k, int box_rows);
 // 2-D bf16 tensor map over the [rows][ldc] output (cols used), box 32 rows x 64
 // columns, 128-byte swizzle: the TMA-store epilogue's map.
 bool make_store_map(CUtensorMap* m, void* base, int64_t rows, int cols, int ldc);
@@ -297,9 +299,16 @@ moe_status launch_gemm_tc2(int epi, const CUtensorMap& ma, const CUtensorMap& mb
                            const CUtensorMap& mc, const moe::TcArgs& args, int64_t max_rows, int groups_bound,
                            cudaStream_t s);
 
+// The swapped-operand SM-pair kernel (gemm_swap.cu), same arguments as
+// launch_gemm_tc; SwiGLU and plain-store epilogues, bf16 only.
+moe_status launch_gemm_swap(int epi, const void* a, const void* b, const void* b2, const int32_t* offsets,
+                            int groups, int max_rows, int nout, int k, void* c, int ldc, int32_t* hdr,
+                            cudaStream_t s, const void* sb, const void* sb2, const void* sa, int sa_rows);
+
 // 0: choose per launch (SM pairs for the store / fp32 epilogues when the
-//    groups average >= 512 rows);
-// 1: single-SM tiles only; 2: SM-pair tiles only.
+//    groups average >= 512 rows, single-SM tiles otherwise);
+// 1: single-SM tiles only; 2: SM-pair tiles only; 3: swapped-operand SM-pair
+//    tiles for the expert GEMMs (the router's fp32 logits keep 0's choice).
 void set_tc_pairing(int mode);
 int tc_pairing();
 }  // namespace moe_host

@@ -104,9 +104,9 @@ def test_host_validation_before_any_launch():
     assert st == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_set_wait_timeout_ns(-1) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_check_device_error(None, 0, None, None) == moe.MOE_ERR_INVALID_ARG
-    for mode in (-1, 3, 1 << 20):
+    for mode in (-1, 4, 1 << 20):
         assert lib.moe_set_gemm_tiling(mode) == moe.MOE_ERR_INVALID_ARG
-    for mode in (1, 2, 0):  # accepted; host state only, no launch
+    for mode in (1, 2, 3, 0):  # accepted; host state only, no launch
         assert lib.moe_set_gemm_tiling(mode) == moe.MOE_OK
 
 
