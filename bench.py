@@ -64,12 +64,15 @@ def _dist():
     return ws, rank, local
 
 
+GEMM_SOURCES = ("gemm_tc.cu", "gemm_tc2.cu", "gemm_swap.cu", "tcgen05.cuh", "tcgen05_pair.cuh")
+
+
 def _kernel_sha():
-    """sha256 prefix of the code of the single-SM grouped GEMM kernel: its two
-    source files with `//` comments, trailing blanks and empty lines removed, so
-    that a comment edit does not retire a traffic figure."""
+    """sha256 prefix of the code of the grouped GEMM kernels: their source
+    files with `//` comments, trailing blanks and empty lines removed, so that a
+    comment edit does not retire a traffic figure."""
     h = hashlib.sha256()
-    for name in ("gemm_tc.cu", "tcgen05.cuh"):
+    for name in GEMM_SOURCES:
         with open(os.path.join(ROOT, "sparse_mixture_experts_rmsnorm_b200", "csrc", name), encoding="utf-8") as f:
             for line in f:
                 code = line.split("//", 1)[0].rstrip()
@@ -211,6 +214,7 @@ def whole_job_tokens_per_s(tokens_per_rank: int, world: int, ms_per_step: float)
 
 
 def run_native(args):
+    import numpy as np
     import torch
     import torch.distributed as dist
 
@@ -393,7 +397,17 @@ def run_native(args):
         shared_launches = 2 if cfg.d_ff_shared > 0 and not fb["shared_folded"] else 0
         chunks = -(-cfg.n_tokens * cfg.top_k // 256)
         permute_launches = 1 if chunks <= 32 and 4 * cfg.n_experts * (chunks + 32) <= 96 * 1024 else 3
-        launches = 1 + int(router_tc) + 1 + permute_launches + 1 + 2 + shared_launches + 1
+        # the grouped down projection of groups averaging >= 512 rows launches
+        # both tilings (the device keeps one of them from the group sizes)
+        # unless the swapped-operand kernel takes it (>= 64 rows a group, H % 64 == 0)
+        cap = int(math.floor(float(np.float32(cfg.capacity_factor)) * cfg.n_tokens * cfg.top_k / cfg.n_experts)) \
+            if cfg.capacity_factor > 0 else cfg.n_tokens * cfg.top_k
+        layout_rows = min(cfg.n_tokens * cfg.top_k, cfg.n_experts * cap)
+        groups = cfg.n_experts + int(fb["shared_folded"])
+        rows_per_group = (layout_rows + (cfg.n_tokens if fb["shared_folded"] else 0)) // groups
+        swap_down = cfg.dtype == "bf16" and args.tiling in (0, 3) and rows_per_group >= 64 and cfg.d_ff % 64 == 0
+        down_both = cfg.dtype == "bf16" and args.tiling == 0 and rows_per_group >= 512 and not swap_down
+        launches = 1 + int(router_tc) + 1 + permute_launches + 1 + 2 + int(down_both) + shared_launches + 1
         line = {
             "metric": METRIC, "value": round(whole_job_tokens_per_s(cfg.n_tokens, world, ms), 1), "unit": UNIT,
             "n_gpus": world,

@@ -15,12 +15,19 @@
 // top-8): there each weight tile is streamed from HBM once, by one SM pair,
 // while the expert's rows (a few MB) stay in L2 across its weight tiles.
 //
+// Loads: every operand comes through a 3-D view of its row-major [rows][K]
+// matrix, {64 columns, rows, K / 64 k-blocks} with the k-block stride 128
+// bytes, so that ONE TMA instruction brings S_KB consecutive k-blocks of a
+// box of rows (the views need K % 64 == 0).  A stage holds S_KB k-blocks; per
+// stage each CTA issues one weight load and one load of its half of the
+// chunk's rows, the latter through the map whose box is exactly that many
+// rows (16 maps, 8 .. 128 rows).  TMA instructions are issued at a limited
+// rate per SM, and one or two of them per k-block left the tensor pipe
+// waiting; two per S_KB k-blocks do not.
+//
 // Roles (192 threads per CTA, clusters of two; as in gemm_tc2.cu):
-//   warp 0      TMA producer in both CTAs: this CTA's 128 weight rows
-//               (SwiGLU: 64 gate rows then the 64 up rows of the same hidden
-//               units) and its half of the chunk's rows, in boxes of 128, 64,
-//               32, 16 and 8 rows; 6-stage ring of 32 KiB; the loads complete
-//               on the even CTA's full barrier;
+//   warp 0      TMA producer in both CTAs; 3-stage ring of 64 KiB; the loads
+//               complete on the even CTA's full barrier;
 //   warp 1      TMEM allocation (512 columns, cta_group::2); in the even CTA
 //               lane 0 issues M = 256, N = rows of the chunk rounded to 16,
 //               K = 16 MMAs into one of two 256-column accumulators and
@@ -29,10 +36,14 @@
 //               column = output row.  Each warp reads 32 x 32 blocks; lanes
 //               trade one value with their neighbour so that each store
 //               writes two adjacent bf16 columns of one output row.  For
-//               SwiGLU the warps holding up rows (lanes 64..127) pass their
-//               fp32 blocks through shared memory to the warps holding the
-//               gate rows of the same hidden units, which apply
-//               silu(gate) * up and store.
+//               SwiGLU the even CTA holds the gate rows and the odd CTA the up
+//               rows of the same 128 hidden units.  Of every 32 output rows
+//               the even CTA finishes the first 16 and the odd CTA the last
+//               16: each warp writes the other 16 columns of its fp32 block
+//               into its partner warp's shared memory in the other CTA
+//               (distributed shared memory, two buffers per warp), takes the
+//               partner's values for its own 16, applies silu(gate) * up and
+//               stores.
 // Tiles run group by group; within a group, chunks in runs of eight share
 // the walk over the weight tiles, so the SM pairs that hold one weight tile's
 // chunks run at the same time.  No TMA load uses cluster multicast.  Every
@@ -47,22 +58,25 @@
 
 namespace moe {
 
-constexpr int S_STAGES = 6;
-constexpr int S_A_BYTES = 128 * TC_BK * 2;           // 16 KiB: this CTA's 128 weight rows
-constexpr int S_B_BYTES = 128 * TC_BK * 2;           // 16 KiB: up to 128 rows of the chunk
-constexpr int S_STAGE_BYTES = S_A_BYTES + S_B_BYTES;  // 32 KiB
-constexpr int S_XCH_BYTES = 32 * 32 * 4;              // one 32 x 32 fp32 block of up values
-constexpr int S_SMEM_BYTES = S_STAGES * S_STAGE_BYTES + 4 * S_XCH_BYTES + 1024;
+constexpr int S_KB = 2;                                // k-blocks per stage (per TMA instruction)
+constexpr int S_STAGES = 3;
+constexpr int S_KBLK_BYTES = 128 * TC_BK * 2;         // one k-block of 128 rows: 16 KiB
+constexpr int S_A_BYTES = S_KB * S_KBLK_BYTES;        // this CTA's 128 weight rows
+constexpr int S_B_BYTES = S_KB * S_KBLK_BYTES;        // up to 128 rows of the chunk
+constexpr int S_STAGE_BYTES = S_A_BYTES + S_B_BYTES;  // 64 KiB
+constexpr int S_XCH_PITCH = 20;                       // words per row of an exchange block (16 + pad)
+constexpr int S_XCH_BYTES = 32 * S_XCH_PITCH * 4;     // one warp's 32 rows x 16 fp32 columns
+constexpr int S_SMEM_BYTES = S_STAGES * S_STAGE_BYTES + 8 * S_XCH_BYTES + 1024;  // 4 warps x 2 buffers
 constexpr int S_THREADS = 192;
 constexpr int S_CHUNK = 256;  // most rows of a group in one tile (the MMA's largest N)
 constexpr int S_RUN = 8;      // chunks that walk a group's weight tiles together
-constexpr int S_BOXES = 5;    // row boxes of 128, 64, 32, 16 and 8 rows
+constexpr int S_XMAPS = 16;   // row boxes of 8, 16, ..., 128 rows
 
 struct SwapMaps {
-  CUtensorMap w[2];            // routed weights: gate and up (64-row boxes) or down (128-row box, w[1] = w[0])
-  CUtensorMap ws[2];           // the folded shared expert's weights, the same boxes
-  CUtensorMap x[S_BOXES];      // the rows: boxes of 128 >> i rows
-  CUtensorMap xs[S_BOXES];     // the shared group's rows when they come from their own tensor
+  CUtensorMap w[2];            // routed weights: gate and up (SwiGLU) or down (w[1] = w[0]); 128-row boxes
+  CUtensorMap ws[2];           // the folded shared expert's weights
+  CUtensorMap x[S_XMAPS];      // the rows: x[i] has boxes of 8 (i + 1) rows
+  CUtensorMap xs[S_XMAPS];     // the shared group's rows when they come from their own tensor
 };
 
 struct SwapArgs {
@@ -70,7 +84,7 @@ struct SwapArgs {
   int groups;
   int max_rows;
   int nout;          // output columns per group (H or d)
-  int K;
+  int K;             // a multiple of 64
   int n_o;           // weight tiles per group: ceil(H / 128) (SwiGLU) or ceil(d / 256)
   void* C;
   int ldc;
@@ -134,32 +148,78 @@ __device__ __forceinline__ SwapTile swap_decode(int t, const int* prefix, const 
   return tl;
 }
 
+// TMA load of S_KB k-blocks of a box of rows through a 3-D view, into this
+// CTA's shared memory, completing on the even CTA's barrier; no multicast.
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar_cluster, int row,
+                                                 int kb) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+      "%4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(0), "r"(row), "r"(kb)
+      : "memory");
+}
+
+// Wait on a barrier that the other CTA of the pair arrives on (acquire at
+// cluster scope), with the bounded-wait rules of mbar_wait_bounded.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Warp-uniform bounded wait: lane 0 waits with the bound, the outcome goes to
 // every lane, and each lane then observes the completed phase itself (which
 // returns at once: the phase cannot move on without this warp).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const SwapArgs& a, volatile int* abort,
-                                          int site) {
+                                          int site, bool cluster_scope) {
   bool ok = true;
-  if (lane_id() == 0) ok = mbar_wait_bounded(bar, parity, a.wait_ns, abort, a.hdr, KID_GEMM_TC, site);
+  if (lane_id() == 0) {
+    if (cluster_scope) {
+      ok = mbar_try_wait_cluster(bar, parity);
+      if (!ok) {
+        const uint64_t t0 = global_timer_ns();
+        for (uint32_t polls = 1; !(ok = mbar_try_wait_cluster(bar, parity)); ++polls) {
+          if ((polls & 63u) == 0u) {
+            if (*abort) break;
+            if (global_timer_ns() - t0 >= a.wait_ns) {
+              record_error(a.hdr, MOE_ERR_DEVICE_TIMEOUT, KID_GEMM_TC, blockIdx.x, site);
+              *abort = 1;
+              break;
+            }
+          }
+        }
+      }
+    } else {
+      ok = mbar_wait_bounded(bar, parity, a.wait_ns, abort, a.hdr, KID_GEMM_TC, site);
+    }
+  }
   ok = __shfl_sync(0xffffffffu, ok, 0);
   if (ok)
-    for (int i = 0; i < (1 << 20) && !mbar_try_wait(bar, parity); ++i) {
-    }
+    for (int i = 0; i < (1 << 20); ++i)
+      if (cluster_scope ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) break;
   return ok;
 }
 
-// Store 32 accumulator columns of this lane's output column `col` (lane =
-// column; the block is rows row0 .. row0 + 31 of C, the first `valid` of them
-// real).  Neighbouring lanes trade one value, so each lane stores two adjacent
-// bf16 columns of one row: the even lane of a pair rows j, the odd lane rows
-// j + 1.  nout is a multiple of 8, so a pair is inside or outside it whole.
+// Store ROWS accumulator columns of this lane's output column `col` (lane =
+// column; the block is rows row0 .. row0 + ROWS - 1 of C, the first `valid` of
+// them real).  Neighbouring lanes trade one value, so each lane stores two
+// adjacent bf16 columns of one row: the even lane of a pair rows j, the odd
+// lane rows j + 1.  nout is a multiple of 8, so a pair is inside or outside
+// it whole.
+template <int ROWS>
 __device__ __forceinline__ void store_cols_bf16x2(bf16* C, int ldc, int row0, int valid, int col, int nout,
-                                                  const float (&v)[32]) {
+                                                  const float (&v)[ROWS]) {
   const bool odd = lane_id() & 1;
   const int c = odd ? col - 1 : col;
   const bool col_ok = c < nout;
 #pragma unroll
-  for (int j = 0; j < 32; j += 2) {
+  for (int j = 0; j < ROWS; j += 2) {
     const float send = odd ? v[j] : v[j + 1];
     const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
     const int r = odd ? j + 1 : j;
@@ -180,8 +240,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
   __shared__ __align__(8) uint64_t empty_bar[S_STAGES];
   __shared__ __align__(8) uint64_t tfull_bar[2];
   __shared__ __align__(8) uint64_t tempty_bar[2];        // used in the even CTA
-  __shared__ __align__(8) uint64_t xfull_bar[2][2];      // SwiGLU: up block of warp pair p, buffer b, written
-  __shared__ __align__(8) uint64_t xempty_bar[2][2];     //         ... and read
+  __shared__ __align__(8) uint64_t xfull_bar[4][2];      // SwiGLU: the partner's block for warp q, buffer b, arrived
+  __shared__ __align__(8) uint64_t xempty_bar[4][2];     //         ... this CTA's block in the partner has been read
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
@@ -208,11 +268,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
       mbar_init(&tempty_bar[b], 8);  // 4 epilogue warps in each CTA
-      for (int p = 0; p < 2; ++p) {
-        mbar_init(&xfull_bar[p][b], 32);
-        mbar_init(&xempty_bar[p][b], 32);
-      }
     }
+    for (int q = 0; q < 4; ++q)
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&xfull_bar[q][b], 32);   // every lane of the partner warp
+        mbar_init(&xempty_bar[q][b], 32);
+      }
     mbar_init(&drain_bar, 1);
     fence_barrier_init();
   }
@@ -228,13 +289,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_sh;
   const int total_tiles = prefix_sh[G];
-  const int nk = (args.K + TC_BK - 1) / TC_BK;
+  const int nk = args.K / TC_BK;
+  const int n_stage_tiles = (nk + S_KB - 1) / S_KB;  // stages per tile
 
   if (warp == 0) {
     // ======================= TMA producer (both CTAs) =======================
     if (lane == 0) {
-      for (int i = 0; i < 2; ++i) tma_prefetch_map(&maps.w[i]);
-      for (int i = 0; i < S_BOXES; ++i) tma_prefetch_map(&maps.x[i]);
+      // SwiGLU: the even CTA loads gate rows, the odd CTA the up rows of the same units
+      const int wsel = (EPI == moe_host::EPI_SWIGLU) ? (int)rank : 0;
+      tma_prefetch_map(&maps.w[wsel]);
       int stage = 0;
       uint32_t phase = 0;
       long issued = 0;
@@ -242,17 +305,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
       for (int t = first; t < total_tiles && ok; t += step) {
         const SwapTile tl = swap_decode(t, prefix_sh, offs_sh, G, args.n_o);
         const bool sh = tl.group == args.shared_group;  // the folded shared expert has its own weights
-        const CUtensorMap* w0 = sh ? &maps.ws[0] : &maps.w[0];
-        const CUtensorMap* w1 = sh ? &maps.ws[1] : &maps.w[1];
+        const CUtensorMap* wm = sh ? &maps.ws[wsel] : &maps.w[wsel];
         const bool own_rows = sh && args.shared_a;       // ... and may read its rows from xn, from row 0
-        const CUtensorMap* xm = own_rows ? maps.xs : maps.x;
         const int half = tl.n >> 1;                      // rows of the chunk in each CTA (8 .. 128)
+        const CUtensorMap* xm = own_rows ? &maps.xs[half / 8 - 1] : &maps.x[half / 8 - 1];
         const int x_row = (own_rows ? tl.row0 - offs_sh[tl.group] : tl.row0) + (int)rank * half;
         const int w_base = sh ? 0 : tl.group * args.nout;
-        const int w_row = EPI == moe_host::EPI_SWIGLU ? w_base + tl.o * 128 + (int)rank * 64
-                                                      : w_base + tl.o * 256 + (int)rank * 128;
-        const uint32_t tx = 2u * (uint32_t)(S_A_BYTES + half * TC_BK * 2);
-        for (int kb = 0; kb < nk; ++kb) {
+        const int w_row = EPI == moe_host::EPI_SWIGLU ? w_base + tl.o * 128 : w_base + tl.o * 256 + (int)rank * 128;
+        const uint32_t tx = 2u * (uint32_t)(S_A_BYTES + S_KB * half * TC_BK * 2);
+        for (int ks = 0; ks < n_stage_tiles; ++ks) {
           if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
                                  SITE_EMPTY)) {
             ok = false;
@@ -260,30 +321,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
           }
           const uint32_t sa = smem_base + stage * S_STAGE_BYTES;
           const uint32_t full_leader = map_to_rank(&full_bar[stage], 0);
-          const int kc = kb * TC_BK;
           if (leader) mbar_arrive_expect_tx(&full_bar[stage], tx);
-          if (EPI == moe_host::EPI_SWIGLU) {
-            tma_load_2d_pair(sa, w0, full_leader, kc, w_row);                   // 64 gate rows
-            tma_load_2d_pair(sa + S_A_BYTES / 2, w1, full_leader, kc, w_row);   // 64 up rows
-          } else {
-            tma_load_2d_pair(sa, w0, full_leader, kc, w_row);                   // 128 weight rows
-          }
-          // this CTA's rows of the chunk, in boxes of 128 or 64 / 32 / 16 / 8 rows
-          uint32_t dst = sa + S_A_BYTES;
-          if (half == 128) {
-            tma_load_2d_pair(dst, &xm[0], full_leader, kc, x_row);
-          } else {
-            int r = x_row;
-#pragma unroll
-            for (int i = 1; i < S_BOXES; ++i) {
-              const int h = 128 >> i;
-              if (half & h) {
-                tma_load_2d_pair(dst, &xm[i], full_leader, kc, r);
-                dst += (uint32_t)(h * TC_BK * 2);
-                r += h;
-              }
-            }
-          }
+          tma_load_3d_pair(sa, wm, full_leader, w_row, ks * S_KB);
+          tma_load_3d_pair(sa + S_A_BYTES, xm, full_leader, x_row, ks * S_KB);
           ++issued;
           if (++stage == S_STAGES) {
             stage = 0;
@@ -317,12 +357,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
       for (int t = first; t < total_tiles && ok; t += step) {
         const SwapTile tl = swap_decode(t, prefix_sh, offs_sh, G, args.n_o);
         const uint32_t idesc = tc_idesc(256, tl.n);
+        const uint32_t b_kblk = (uint32_t)((tl.n >> 1) * TC_BK * 2);  // bytes of one k-block of this CTA's rows
         if (!mbar_wait_bounded(&tempty_bar[buf], bphase ^ 1u, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
                                SITE_TMEM_EMPTY))
           break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(buf * 256);
-        for (int kb = 0; kb < nk; ++kb) {
+        for (int ks = 0; ks < n_stage_tiles; ++ks) {
           if (!mbar_wait_bounded(&full_bar[stage], phase, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
                                  SITE_FULL)) {
             ok = false;
@@ -330,11 +371,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
           }
           tc_fence_after();
           const uint32_t sa = smem_base + stage * S_STAGE_BYTES;
-          const uint64_t adesc = sw128_desc(sa);
-          const uint64_t bdesc = sw128_desc(sa + S_A_BYTES);
+          const int kb_n = min(S_KB, nk - ks * S_KB);  // k-blocks of this stage inside K
+          for (int j = 0; j < kb_n; ++j) {
+            const uint64_t adesc = sw128_desc(sa + (uint32_t)(j * S_KBLK_BYTES));
+            const uint64_t bdesc = sw128_desc(sa + S_A_BYTES + (uint32_t)j * b_kblk);
 #pragma unroll
-          for (int kk = 0; kk < TC_BK / 16; ++kk)
-            tc2_mma(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc, (kb | kk) != 0);
+            for (int kk = 0; kk < TC_BK / 16; ++kk)
+              tc2_mma(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), idesc, (ks | j | kk) != 0);
+          }
           tc2_commit_both(&empty_bar[stage]);
           if (++stage == S_STAGES) {
             stage = 0;
@@ -356,17 +400,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
   } else {
     // ======================= epilogue (warps 2..5, both CTAs) =======================
     const int quarter = warp & 3;  // TMEM lanes 32 * quarter .. + 31
-    const int pair = quarter & 1;  // SwiGLU: gate quarter `pair`, up quarter `pair + 2`
-    const bool up_warp = EPI == moe_host::EPI_SWIGLU && quarter >= 2;
-    const uint32_t xch = smem_base + S_STAGES * S_STAGE_BYTES;
+    const uint32_t peer = rank ^ 1u;
+    // SwiGLU exchange: buffer b of this warp's row `lane` (16 fp32), here and in the partner CTA
+    const uint32_t xrow = smem_base + S_STAGES * S_STAGE_BYTES + (uint32_t)(quarter * 2 * S_XCH_BYTES) +
+                          (uint32_t)(lane * S_XCH_PITCH * 4);
     bf16* C = reinterpret_cast<bf16*>(args.C);
     int buf = 0;
     uint32_t bphase = 0;
-    uint32_t xcnt = 0;  // SwiGLU blocks this warp pair has passed so far
+    uint32_t xi = 0;  // SwiGLU: 32-column blocks this warp has handled (buffer xi & 1, phase (xi >> 1) & 1)
     bool ok = true;
     for (int t = first; t < total_tiles && ok; t += step) {
       const SwapTile tl = swap_decode(t, prefix_sh, offs_sh, G, args.n_o);
-      if (!warp_wait(&tfull_bar[buf], bphase, args, &abort_flag, SITE_TMEM_FULL)) break;
+      if (!warp_wait(&tfull_bar[buf], bphase, args, &abort_flag, SITE_TMEM_FULL, false)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * 256);
       if (EPI == moe_host::EPI_STORE) {
@@ -379,43 +424,60 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(a[i]);
-          store_cols_bf16x2(C, args.ldc, tl.row0 + c0, tl.rows - c0, col, args.nout, v);
+          store_cols_bf16x2<32>(C, args.ldc, tl.row0 + c0, tl.rows - c0, col, args.nout, v);
         }
       } else {
-        const int col = tl.o * 128 + (int)rank * 64 + pair * 32 + lane;  // hidden unit
+        const int col = tl.o * 128 + quarter * 32 + lane;  // hidden unit
 #pragma unroll 1
-        for (int c0 = 0; c0 < tl.rows; c0 += 32, ++xcnt) {
-          const int b = (int)(xcnt & 1u);
-          const uint32_t ph = (xcnt >> 1) & 1u;
-          const uint32_t blk = xch + (uint32_t)((pair * 2 + b) * S_XCH_BYTES) + (uint32_t)lane * 4u;
-          uint32_t a[32];
+        for (int c0 = 0; c0 < tl.rows; c0 += 32, ++xi) {
+          const int b = (int)(xi & 1u);
+          const uint32_t ph = (xi >> 1) & 1u;
+          const uint32_t xb = xrow + (uint32_t)(b * S_XCH_BYTES);
+          uint32_t a[32];  // gate (even CTA) or up (odd CTA) of 32 output rows
           MOE_TMEM_LD32(tbase + c0, a);
           tmem_wait_ld();
-          if (up_warp) {
-            // hand the up values (fp32, [column][lane]) to the gate warp
-            if (!warp_wait(&xempty_bar[pair][b], ph ^ 1u, args, &abort_flag, SITE_XEMPTY)) {
-              ok = false;
-              break;
-            }
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              asm volatile("st.shared.b32 [%0], %1;" ::"r"(blk + (uint32_t)(j * 128)), "r"(a[j]) : "memory");
-            mbar_arrive(&xfull_bar[pair][b]);
-          } else {
-            if (!warp_wait(&xfull_bar[pair][b], ph, args, &abort_flag, SITE_XFULL)) {
-              ok = false;
-              break;
-            }
-            float v[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              uint32_t u;
-              asm volatile("ld.shared.b32 %0, [%1];" : "=r"(u) : "r"(blk + (uint32_t)(j * 128)) : "memory");
-              v[j] = __fmul_rn(silu_tc(__uint_as_float(a[j])), __uint_as_float(u));
-            }
-            mbar_arrive(&xempty_bar[pair][b]);
-            store_cols_bf16x2(C, args.ldc, tl.row0 + c0, tl.rows - c0, col, args.nout, v);
+          // the partner finishes the other 16 rows: send it this CTA's values of those
+          if (!warp_wait(&xempty_bar[quarter][b], ph ^ 1u, args, &abort_flag, SITE_XEMPTY, true)) {
+            ok = false;
+            break;
           }
+          // rows 0..15 go to (or stay with) the even CTA, rows 16..31 the odd one
+          uint32_t snd[16], own[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            snd[j] = leader ? a[16 + j] : a[j];
+            own[j] = leader ? a[j] : a[16 + j];
+          }
+          const uint32_t dst = map_to_rank_addr(xb, peer);
+#pragma unroll
+          for (int j = 0; j < 16; j += 4)
+            asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + (uint32_t)(j * 4)),
+                         "r"(snd[j]), "r"(snd[j + 1]), "r"(snd[j + 2]), "r"(snd[j + 3])
+                         : "memory");
+          mbar_arrive_cluster(map_to_rank(&xfull_bar[quarter][b], peer));
+          // ... and take the partner's values of this CTA's 16 rows
+          if (!warp_wait(&xfull_bar[quarter][b], ph, args, &abort_flag, SITE_XFULL, true)) {
+            ok = false;
+            break;
+          }
+          const int mine = (int)rank * 16;
+          float v[16];
+#pragma unroll
+          for (int j = 0; j < 16; j += 4) {
+            uint32_t u[4];
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
+                         : "r"(xb + (uint32_t)(j * 4))
+                         : "memory");
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float mv = __uint_as_float(own[j + i]), other = __uint_as_float(u[i]);
+              const float g = leader ? mv : other, up = leader ? other : mv;
+              v[j + i] = __fmul_rn(silu_tc(g), up);
+            }
+          }
+          mbar_arrive_cluster(map_to_rank(&xempty_bar[quarter][b], peer));
+          store_cols_bf16x2<16>(C, args.ldc, tl.row0 + c0 + mine, tl.rows - c0 - mine, col, args.nout, v);
         }
         if (!ok) break;
       }
@@ -441,6 +503,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
 }  // namespace moe
 
 namespace moe_host {
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();  // gemm_tc.cu
+
+// 3-D view {64 columns, rows, k / 64 k-blocks} of a row-major bf16 [rows][k]
+// matrix (k % 64 == 0), the k-block stride 128 bytes: a box of `box_rows`
+// rows and S_KB k-blocks, 128-byte swizzle, zero fill outside the matrix.
+static bool make_kblock_map(CUtensorMap* m, const void* base, int64_t rows, int k, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)moe::TC_BK, (cuuint64_t)rows, (cuuint64_t)(k / moe::TC_BK)};
+  cuuint64_t strides[2] = {(cuuint64_t)k * 2, (cuuint64_t)moe::TC_BK * 2};
+  cuuint32_t box[3] = {(cuuint32_t)moe::TC_BK, (cuuint32_t)box_rows, (cuuint32_t)moe::S_KB};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
 
 // Clusters of two that can be resident at once (one CTA per SM), per device.
 template <int EPI>
@@ -476,17 +556,19 @@ static moe_status launch_swap_t(const moe::SwapMaps& maps, const moe::SwapArgs& 
   return launch_status();
 }
 
+bool swap_supported(int epi, int nout, int k, int ldc) {
+  return epi != EPI_F32 && k % moe::TC_BK == 0 && nout % 8 == 0 && ldc % 8 == 0;
+}
+
 moe_status launch_gemm_swap(int epi, const void* a, const void* b, const void* b2, const int32_t* offsets,
                             int groups, int max_rows, int nout, int k, void* c, int ldc, int32_t* hdr,
                             cudaStream_t s, const void* sb, const void* sb2, const void* sa, int sa_rows) {
   if (max_rows == 0 || nout == 0 || groups == 0) return MOE_OK;
-  if (epi == EPI_F32 || groups > moe::TC_MAX_GROUPS || (k % 8) != 0 || (nout % 8) != 0 || (ldc % 8) != 0)
-    return MOE_ERR_UNSUPPORTED;
+  if (!swap_supported(epi, nout, k, ldc) || groups > moe::TC_MAX_GROUPS) return MOE_ERR_UNSUPPORTED;
   if (((uintptr_t)a | (uintptr_t)b | (uintptr_t)(b2 ? b2 : b) | (uintptr_t)(sb ? sb : b) |
        (uintptr_t)(sb2 ? sb2 : b) | (uintptr_t)(sa ? sa : a) | (uintptr_t)c) % 16 != 0)
     return MOE_ERR_UNSUPPORTED;
   const bool swiglu = epi == EPI_SWIGLU;
-  const int wbox = swiglu ? 64 : 128;
   moe::SwapMaps maps;
   // the routed weights hold one [nout][k] block per routed group only; a
   // folded shared expert (the last group) has its own tensors
@@ -494,21 +576,21 @@ moe_status launch_gemm_swap(int epi, const void* a, const void* b, const void* b
   const int64_t w_rows = std::max<int64_t>((int64_t)routed_groups * nout, 1);
   const bool shared_a = sb != nullptr && offsets && sa != nullptr && sa_rows > 0;
   const int64_t x_rows = shared_a ? std::max<int64_t>((int64_t)max_rows - sa_rows, 1) : max_rows;
-  if (!make_tc_map_rows(&maps.w[0], b, w_rows, k, wbox)) return MOE_ERR_CUDA;
+  if (!make_kblock_map(&maps.w[0], b, w_rows, k, 128)) return MOE_ERR_CUDA;
   maps.w[1] = maps.w[0];
-  if (swiglu && !make_tc_map_rows(&maps.w[1], b2, w_rows, k, wbox)) return MOE_ERR_CUDA;
+  if (swiglu && !make_kblock_map(&maps.w[1], b2, w_rows, k, 128)) return MOE_ERR_CUDA;
   if (sb != nullptr) {
-    if (!make_tc_map_rows(&maps.ws[0], sb, nout, k, wbox)) return MOE_ERR_CUDA;
+    if (!make_kblock_map(&maps.ws[0], sb, nout, k, 128)) return MOE_ERR_CUDA;
     maps.ws[1] = maps.ws[0];
-    if (swiglu && !make_tc_map_rows(&maps.ws[1], sb2, nout, k, wbox)) return MOE_ERR_CUDA;
+    if (swiglu && !make_kblock_map(&maps.ws[1], sb2, nout, k, 128)) return MOE_ERR_CUDA;
   } else {
     maps.ws[0] = maps.w[0];
     maps.ws[1] = maps.w[1];
   }
-  for (int i = 0; i < moe::S_BOXES; ++i) {
-    if (!make_tc_map_rows(&maps.x[i], a, x_rows, k, 128 >> i)) return MOE_ERR_CUDA;
+  for (int i = 0; i < moe::S_XMAPS; ++i) {
+    if (!make_kblock_map(&maps.x[i], a, x_rows, k, 8 * (i + 1))) return MOE_ERR_CUDA;
     if (shared_a) {
-      if (!make_tc_map_rows(&maps.xs[i], sa, sa_rows, k, 128 >> i)) return MOE_ERR_CUDA;
+      if (!make_kblock_map(&maps.xs[i], sa, sa_rows, k, 8 * (i + 1))) return MOE_ERR_CUDA;
     } else {
       maps.xs[i] = maps.x[i];
     }

@@ -79,6 +79,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     offs_sh[i] = args.offsets ? args.offsets[i] : (i == 0 ? 0 : args.max_rows);
   if (threadIdx.x == 0) abort_flag = 0;
   __syncthreads();
+  if (args.pick != 0) {
+    // both tilings were launched: the one not picked for these groups ends here
+    __shared__ int picked_sh;
+    if (warp == 0) {
+      const bool pairs = pairs_picked(offs_sh, G, args.n_tiles, args.pick_pairs, args.pick_ctas);
+      if (lane == 0) picked_sh = pairs ? 2 : 1;
+    }
+    __syncthreads();
+    if (picked_sh != args.pick) return;
+  }
   if (warp == 0) build_prefix<TC_BM>(offs_sh, prefix_sh, G, args.n_tiles);
   if (threadIdx.x == 0) {
     for (int s = 0; s < TC_STAGES; ++s) {
@@ -281,7 +291,7 @@ namespace moe_host {
 
 // The driver's tensor-map encoder, looked up once (a function-local static, so the first calls of several host
 // threads are safe); nullptr when the driver does not export it.
-static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -294,7 +304,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
 }
 
 bool make_store_map(CUtensorMap* m, void* base, int64_t rows, int cols, int ldc) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode();
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)ldc * 2};
@@ -309,7 +319,7 @@ bool make_store_map(CUtensorMap* m, void* base, int64_t rows, int cols, int ldc)
 bool make_tc_map(CUtensorMap* m, const void* base, int64_t rows, int k) { return make_tc_map_rows(m, base, rows, k, 128); }
 
 bool make_tc_map_rows(CUtensorMap* m, const void* base, int64_t rows, int k, int box_rows) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = get_encode();
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (enc == nullptr) return false;
   cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)k * 2};
@@ -385,6 +395,9 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
   args.n_tiles = (nout + args.out_cols - 1) / args.out_cols;
   args.narrow = 0;
   args.tma_store = 0;
+  args.pick = 0;
+  args.pick_pairs = 1;
+  args.pick_ctas = 1;
   args.C = c;
   args.ldc = ldc;
   args.hdr = hdr;
@@ -404,9 +417,19 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
   const int rows_per_group = max_rows / (offsets ? groups : 1);
   const int forced = tc_pairing();
   // Operands swapped on SM pairs (gemm_swap.cu): weight rows on M, the
-  // group's rows on N in chunks of at most 256 padded to 16.  Measured slower
-  // than the tilings below on every workload so far, so only on request.
-  if (epi != EPI_F32 && forced == 3)
+  // group's rows on N in chunks of at most 256 padded to 16 (K a multiple of
+  // 64).  Measured on B200 (same box, one run each):
+  //  - the down projection of every prefill-sized workload (groups averaging
+  //    >= 64 rows) is fastest this way: DeepSeek-V3-shaped 2.25 against
+  //    2.47 ms, Mixtral-shaped 0.67 against 0.74 ms (and 0.88 with SM pairs),
+  //    load-imbalance 0.53 against 0.56 ms;
+  //  - the SwiGLU projection only where there are many groups of a few
+  //    hundred rows: DeepSeek-V3-shaped 4.54 against 4.66 ms, but
+  //    Mixtral-shaped (8 groups of 1024) 2.05 against 1.67 ms;
+  //  - decode (2 rows a group) keeps the M = 64 tiles.
+  const bool swap_auto = forced == 0 && offsets != nullptr && rows_per_group >= 64 &&
+                         (epi == EPI_STORE || (epi == EPI_SWIGLU && groups >= 16 && rows_per_group < 512));
+  if ((forced == 3 || swap_auto) && swap_supported(epi, nout, k, ldc))
     return launch_gemm_swap(epi, a, b, b2, offsets, groups, max_rows, nout, k, c, ldc, hdr, s, sb, sb2, sa, sa_rows);
   const int mode = forced == 3 ? 0 : forced;  // the router's fp32 logits: the automatic choice
   // Upper bound on the number of tiles; the exact count lives on the device.
@@ -416,9 +439,15 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
   // 128-column tiles on single SMs instead, twice as many.
   const bool few = epi != EPI_SWIGLU && mode != 2 && nout > 128 && m_tiles * args.n_tiles < sm_count() / 2;
   // Measured on B200: SM pairs help the plain-store epilogue of large groups
-  // (down projection) by a few percent; for the SwiGLU projection the extra
-  // padding of 256-row tiles outweighs the saved operand traffic.
-  if (mode == 2 || (mode == 0 && rows_per_group >= 512 && epi != EPI_SWIGLU && !few))
+  // (down projection) by a few percent when both tilings take the same number
+  // of waves; for the SwiGLU projection the extra padding of 256-row tiles
+  // outweighs the saved operand traffic.  The group sizes live on the device,
+  // so for the grouped down projection both kernels are launched and each
+  // keeps or drops itself from the offsets (pairs_picked); the router's
+  // single group keeps the host rule.
+  const bool pair_rule = mode == 2 || (mode == 0 && rows_per_group >= 512 && epi != EPI_SWIGLU && !few);
+  const bool device_pick = mode == 0 && pair_rule && epi == EPI_STORE && offsets != nullptr;
+  if (pair_rule && !device_pick)
     return launch_gemm_tc2(epi, ma, mb, mb2, msb, msb2, msa, mc, args, max_rows, offsets ? groups : 0, s);
   if (few) {
     args.narrow = 1;
@@ -427,6 +456,14 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
   }
   const int64_t bound = m_tiles * args.n_tiles;
   const int grid = (int)(bound < sm_count() ? bound : sm_count());
+  if (device_pick) {
+    args.pick_pairs = (int)tc2_pairs_launched(epi, max_rows, groups, args.n_tiles);
+    args.pick_ctas = grid;
+    args.pick = 2;
+    const moe_status st = launch_gemm_tc2(epi, ma, mb, mb2, msb, msb2, msa, mc, args, max_rows, groups, s);
+    if (st != MOE_OK) return st;
+    args.pick = 1;
+  }
   if (epi == EPI_SWIGLU) return launch_tc_t<EPI_SWIGLU>(ma, mb, mb2, msb, msb2, msa, mc, args, grid, s);
   if (epi == EPI_STORE) return launch_tc_t<EPI_STORE>(ma, mb, mb2, msb, msb2, msa, mc, args, grid, s);
   return launch_tc_t<EPI_F32>(ma, mb, mb2, msb, msb2, msa, mc, args, grid, s);

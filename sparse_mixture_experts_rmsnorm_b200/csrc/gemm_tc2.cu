@@ -66,6 +66,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(P_THREADS, 1)
     offs_sh[i] = args.offsets ? args.offsets[i] : (i == 0 ? 0 : args.max_rows);
   if (threadIdx.x == 0) abort_flag = 0;
   __syncthreads();
+  if (args.pick != 0) {
+    // both tilings were launched: the one not picked for these groups ends here
+    __shared__ int picked_sh;
+    if (warp == 0) {
+      const bool pairs = pairs_picked(offs_sh, G, args.n_tiles, args.pick_pairs, args.pick_ctas);
+      if (lane == 0) picked_sh = pairs ? 2 : 1;
+    }
+    __syncthreads();
+    if (picked_sh != args.pick) return;
+  }
   if (warp == 0) build_prefix<P_BM>(offs_sh, prefix_sh, G, args.n_tiles);
   if (threadIdx.x == 0) {
     for (int s = 0; s < P_STAGES; ++s) {
@@ -265,6 +275,23 @@ static int resident_pairs() {
   return n;
 }
 
+static int resident_pairs_of(int epi) {
+  if (epi == EPI_SWIGLU) return resident_pairs<EPI_SWIGLU>();
+  if (epi == EPI_STORE) return resident_pairs<EPI_STORE>();
+  return resident_pairs<EPI_F32>();
+}
+
+// Upper bound on the pair tiles (the exact count lives on the device).
+static int64_t pair_tile_bound(int64_t max_rows, int groups_bound, int n_tiles) {
+  return ((max_rows + moe::P_BM - 1) / moe::P_BM + groups_bound) * n_tiles;
+}
+
+int64_t tc2_pairs_launched(int epi, int64_t max_rows, int groups_bound, int n_tiles) {
+  const int64_t bound = pair_tile_bound(max_rows, groups_bound, n_tiles);
+  const int64_t res = resident_pairs_of(epi);
+  return bound < res ? bound : res;
+}
+
 template <int EPI>
 static moe_status launch_tc2_t(const CUtensorMap& ma, const CUtensorMap& mb, const CUtensorMap& mb2,
                                const CUtensorMap& msb, const CUtensorMap& msb2, const CUtensorMap& msa,
@@ -283,9 +310,7 @@ moe_status launch_gemm_tc2(int epi, const CUtensorMap& ma, const CUtensorMap& mb
                            const CUtensorMap& msb, const CUtensorMap& msb2, const CUtensorMap& msa,
                            const CUtensorMap& mc, const moe::TcArgs& args, int64_t max_rows, int groups_bound,
                            cudaStream_t s) {
-  // upper bound on the pair tiles; the exact count lives on the device
-  const int64_t m_pairs = (max_rows + moe::P_BM - 1) / moe::P_BM + groups_bound;
-  const int64_t bound = m_pairs * args.n_tiles;
+  const int64_t bound = pair_tile_bound(max_rows, groups_bound, args.n_tiles);
   if (epi == EPI_SWIGLU) return launch_tc2_t<EPI_SWIGLU>(ma, mb, mb2, msb, msb2, msa, mc, args, bound, s);
   if (epi == EPI_STORE) return launch_tc2_t<EPI_STORE>(ma, mb, mb2, msb, msb2, msa, mc, args, bound, s);
   return launch_tc2_t<EPI_F32>(ma, mb, mb2, msb, msb2, msa, mc, args, bound, s);

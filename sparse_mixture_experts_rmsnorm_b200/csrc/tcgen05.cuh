@@ -34,7 +34,36 @@ struct TcArgs {
   int shared_a;      // 1: that group's A rows come from their own map, from row 0
   int narrow;        // 1: 128-column tiles (one B box, N = 128), plain epilogues only
   int tma_store;     // 1: the plain-store epilogue writes whole warps' blocks through TMA
+  // Tiling picked on the device from the group sizes (both kernels are
+  // launched; the one not picked returns at once): 0 = always run,
+  // 1 = run if single-SM tiles are picked, 2 = run if SM-pair tiles are.
+  int pick;
+  int pick_pairs;    // SM pairs resident for the pair kernel
+  int pick_ctas;     // CTAs of the single-SM kernel
 };
+
+// The device-side tiling choice of the plain-store epilogue (down
+// projection): with persistent CTAs taking tiles in turn, a launch lasts
+// about ceil(tiles / workers) tile times; an SM-pair tile does one SM's
+// share of work about 3 % faster than a single-SM tile (measured on B200),
+// so pairs are picked when 97 * their waves <= 100 * the single-SM waves.
+// Called by one whole warp; every lane returns the same answer.
+__device__ __forceinline__ bool pairs_picked(const int* offs, int groups, int n_tiles, int pairs, int ctas) {
+  int tp = 0, ts = 0;
+  for (int g = lane_id(); g < groups; g += 32) {
+    const int m = offs[g + 1] - offs[g];
+    tp += (m + 255) / 256;
+    ts += (m + 127) / 128;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    tp += __shfl_xor_sync(0xffffffffu, tp, o);
+    ts += __shfl_xor_sync(0xffffffffu, ts, o);
+  }
+  const long wp = ((long)tp * n_tiles + pairs - 1) / pairs;
+  const long wsg = ((long)ts * n_tiles + ctas - 1) / ctas;
+  return 97 * wp <= 100 * wsg;
+}
 
 // ---- PTX wrappers -----------------------------------------------------------
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint64_t* bar, int c0, int c1) {
@@ -300,13 +329,25 @@ moe_status launch_gemm_tc2(int epi, const CUtensorMap& ma, const CUtensorMap& mb
                            cudaStream_t s);
 
 // The swapped-operand SM-pair kernel (gemm_swap.cu), same arguments as
-// launch_gemm_tc; SwiGLU and plain-store epilogues, bf16 only.
+// launch_gemm_tc; SwiGLU and plain-store epilogues, bf16 only, for the shapes
+// swap_supported accepts (K a multiple of 64, nout and ldc multiples of 8).
+bool swap_supported(int epi, int nout, int k, int ldc);
 moe_status launch_gemm_swap(int epi, const void* a, const void* b, const void* b2, const int32_t* offsets,
                             int groups, int max_rows, int nout, int k, void* c, int ldc, int32_t* hdr,
                             cudaStream_t s, const void* sb, const void* sb2, const void* sa, int sa_rows);
 
-// 0: choose per launch (SM pairs for the store / fp32 epilogues when the
-//    groups average >= 512 rows, single-SM tiles otherwise);
+// SM pairs that launch_gemm_tc2 launches for these sizes.
+int64_t tc2_pairs_launched(int epi, int64_t max_rows, int groups_bound, int n_tiles);
+
+// 3: the swapped-operand SM-pair kernel for the expert GEMMs it supports
+//    (the rest, and the router, take 0's choice);
+// 0: choose per launch (the swapped-operand kernel, where it supports the
+//    shape, for the grouped plain store of groups averaging >= 64 rows and
+//    for SwiGLU over 16 or more groups averaging 64 .. 511 rows; single-SM
+//    tiles for the other SwiGLU launches; for the grouped plain store of groups
+//    averaging >= 512 rows both kernels are launched and the device picks
+//    from the group sizes (pairs_picked); the router's single group takes SM
+//    pairs from 512 rows);
 // 1: single-SM tiles only; 2: SM-pair tiles only; 3: swapped-operand SM-pair
 //    tiles for the expert GEMMs (the router's fp32 logits keep 0's choice).
 void set_tc_pairing(int mode);

@@ -12,8 +12,9 @@ import pytest
 
 import moe_inputs as mi
 import oracle
-from parity_helpers import (BF16_REL_RMS, bf16_rel_rms_err, capacity, check_permutation, check_routing,
-                            oracle_outputs, oracle_routing, rel_rms_err, run_gpu_layer, tie_masks, to_np)
+from parity_helpers import (BF16_REL_RMS, bf16_half_ulp, bf16_rel_rms_err, capacity, check_permutation,
+                            check_routing, oracle_outputs, oracle_routing, rel_rms_err, run_gpu_layer, tie_masks,
+                            to_np)
 
 pytestmark = pytest.mark.gpu
 
@@ -86,8 +87,13 @@ def test_config_parity(name):
     err = bf16_rel_rms_err(got, ref_out)
     raw = rel_rms_err(got, ref_out)
     raw_delta = rel_rms_err(got - ref["h"][tokens], ref_out - ref["h"][tokens])
+    # the same beyond-storage error, relative to the layer's contribution out - h
+    delta_rms = float(np.sqrt(np.mean((ref_out - ref["h"][tokens]) ** 2)))
+    bs_delta = float(np.max(np.maximum(np.abs(got - ref_out) - bf16_half_ulp(ref_out), 0.0)) / delta_rms)
     print(f"PARITY {name}: beyond-storage max err/rms(out) = {err:.3e}; raw max|err|/rms(out) = {raw:.3e}; "
-          f"raw max|err| on out-h / rms(out-h) = {raw_delta:.3e}; tokens {tokens.size}, experts covered "
+          f"raw max|err| on out-h / rms(out-h) = {raw_delta:.3e}; beyond-storage max err / rms(out-h) = "
+          f"{bs_delta:.3e}; rms(out) = {np.sqrt(np.mean(ref_out ** 2)):.3f}, rms(out-h) = {delta_rms:.4f}; "
+          f"tokens {tokens.size}, experts covered "
           f"{covered.size} of {E}{' + shared' if cfg.d_ff_shared else ''}, skipped ties {skipped}, "
           f"dropped slots {int((~gpu_keep).sum())}")
     assert err <= BF16_REL_RMS, err

@@ -243,6 +243,22 @@ def test_expert_ffn_tc_single_group_smaller_than_a_tile(torch_cuda, gemm_tiling,
     assert bf16_rel_rms_err(got, ref) <= BF16_REL_RMS
 
 
+@pytest.mark.parametrize("rows,d,H", [
+    # the load-imbalance workload's kept rows per expert: single-SM tiles take
+    # fewer waves at d = 4096 (16 column tiles), so the device picks them
+    ([629, 726, 586, 1280, 565, 766, 343, 615], 4096, 136),
+    # the same groups at d = 256 fit one wave either way: SM pairs are picked
+    ([629, 726, 586, 1280, 565, 766, 343, 615], 256, 136),
+])
+def test_down_projection_tiling_picked_on_the_device(torch_cuda, gemm_tiling, rows, d, H):
+    # groups averaging >= 512 rows with H % 64 != 0 (the swapped-operand kernel
+    # declines): the down projection launches both other tilings and the
+    # device keeps one from the offsets; the output is the oracle's
+    gemm_tiling(0)
+    got, ref = _ffn_case(torch_cuda, rows, d, H, seed=13)
+    assert bf16_rel_rms_err(got, ref) <= BF16_REL_RMS
+
+
 def test_both_tilings_agree_closely(torch_cuda, gemm_tiling):
     # same products, summation order aside
     gemm_tiling(1)
