@@ -232,6 +232,11 @@ __device__ __forceinline__ void store_cols_bf16x2(bf16* C, int ldc, int row0, in
 
 enum { SITE_XFULL = 6, SITE_XEMPTY = 7 };
 
+// silu(z) = z / (1 + e^-z) with the fast exp and divide intrinsics: about 1e-6
+// relative error in fp32, far below the bf16 rounding of the activation that
+// follows; z -> -inf gives -0, z -> +inf gives z.
+__device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.f + __expf(-z)); }
+
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
     gemm_swap_kernel(const __grid_constant__ SwapMaps maps, const SwapArgs args) {
@@ -407,7 +412,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
     bf16* C = reinterpret_cast<bf16*>(args.C);
     int buf = 0;
     uint32_t bphase = 0;
-    uint32_t xi = 0;  // SwiGLU: 32-column blocks this warp has handled (buffer xi & 1, phase (xi >> 1) & 1)
+    uint32_t xi = 0;  // SwiGLU: 32-row blocks this warp has handled (buffer xi & 1, phase (xi >> 1) & 1)
     bool ok = true;
     for (int t = first; t < total_tiles && ok; t += step) {
       const SwapTile tl = swap_decode(t, prefix_sh, offs_sh, G, args.n_o);
@@ -427,57 +432,74 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
           store_cols_bf16x2<32>(C, args.ldc, tl.row0 + c0, tl.rows - c0, col, args.nout, v);
         }
       } else {
+        // Block i of 32 output rows: rows 0..15 are finished by the even CTA,
+        // rows 16..31 by the odd one.  Each warp sends its partner the values
+        // of the partner's rows of block i + 1 before it waits for the
+        // partner's values of block i, so the exchange latency hides behind
+        // a block of work.
         const int col = tl.o * 128 + quarter * 32 + lane;  // hidden unit
-#pragma unroll 1
-        for (int c0 = 0; c0 < tl.rows; c0 += 32, ++xi) {
-          const int b = (int)(xi & 1u);
-          const uint32_t ph = (xi >> 1) & 1u;
-          const uint32_t xb = xrow + (uint32_t)(b * S_XCH_BYTES);
-          uint32_t a[32];  // gate (even CTA) or up (odd CTA) of 32 output rows
-          MOE_TMEM_LD32(tbase + c0, a);
+        const int nblk = (tl.rows + 31) >> 5;
+        uint32_t own[16];  // this CTA's values (gate or up) of its own 16 rows of the current block
+        // send block j (buffer xi & 1 of the partner) and keep this CTA's half of it in own[]
+        auto send_block = [&](int j, uint32_t x) -> bool {
+          uint32_t a[32];
+          MOE_TMEM_LD32(tbase + (uint32_t)(j * 32), a);
           tmem_wait_ld();
-          // the partner finishes the other 16 rows: send it this CTA's values of those
-          if (!warp_wait(&xempty_bar[quarter][b], ph ^ 1u, args, &abort_flag, SITE_XEMPTY, true)) {
-            ok = false;
-            break;
-          }
-          // rows 0..15 go to (or stay with) the even CTA, rows 16..31 the odd one
-          uint32_t snd[16], own[16];
+          const int b = (int)(x & 1u);
+          if (!warp_wait(&xempty_bar[quarter][b], ((x >> 1) & 1u) ^ 1u, args, &abort_flag, SITE_XEMPTY, true))
+            return false;
+          uint32_t snd[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            snd[j] = leader ? a[16 + j] : a[j];
-            own[j] = leader ? a[j] : a[16 + j];
+          for (int i = 0; i < 16; ++i) {
+            snd[i] = leader ? a[16 + i] : a[i];
+            own[i] = leader ? a[i] : a[16 + i];
           }
-          const uint32_t dst = map_to_rank_addr(xb, peer);
+          const uint32_t dst = map_to_rank_addr(xrow + (uint32_t)(b * S_XCH_BYTES), peer);
 #pragma unroll
-          for (int j = 0; j < 16; j += 4)
-            asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + (uint32_t)(j * 4)),
-                         "r"(snd[j]), "r"(snd[j + 1]), "r"(snd[j + 2]), "r"(snd[j + 3])
+          for (int i = 0; i < 16; i += 4)
+            asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + (uint32_t)(i * 4)),
+                         "r"(snd[i]), "r"(snd[i + 1]), "r"(snd[i + 2]), "r"(snd[i + 3])
                          : "memory");
           mbar_arrive_cluster(map_to_rank(&xfull_bar[quarter][b], peer));
-          // ... and take the partner's values of this CTA's 16 rows
-          if (!warp_wait(&xfull_bar[quarter][b], ph, args, &abort_flag, SITE_XFULL, true)) {
+          return true;
+        };
+        if (nblk > 0 && !send_block(0, xi)) {
+          ok = false;
+          break;
+        }
+#pragma unroll 1
+        for (int j = 0; j < nblk; ++j, ++xi) {
+          uint32_t cur[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) cur[i] = own[i];
+          if (j + 1 < nblk && !send_block(j + 1, xi + 1)) {
             ok = false;
             break;
           }
-          const int mine = (int)rank * 16;
+          const int b = (int)(xi & 1u);
+          if (!warp_wait(&xfull_bar[quarter][b], (xi >> 1) & 1u, args, &abort_flag, SITE_XFULL, true)) {
+            ok = false;
+            break;
+          }
+          const uint32_t xb = xrow + (uint32_t)(b * S_XCH_BYTES);
           float v[16];
 #pragma unroll
-          for (int j = 0; j < 16; j += 4) {
+          for (int i = 0; i < 16; i += 4) {
             uint32_t u[4];
             asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                          : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
-                         : "r"(xb + (uint32_t)(j * 4))
+                         : "r"(xb + (uint32_t)(i * 4))
                          : "memory");
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float mv = __uint_as_float(own[j + i]), other = __uint_as_float(u[i]);
+            for (int e = 0; e < 4; ++e) {
+              const float mv = __uint_as_float(cur[i + e]), other = __uint_as_float(u[e]);
               const float g = leader ? mv : other, up = leader ? other : mv;
-              v[j + i] = __fmul_rn(silu_tc(g), up);
+              v[i + e] = __fmul_rn(silu_fast(g), up);
             }
           }
           mbar_arrive_cluster(map_to_rank(&xempty_bar[quarter][b], peer));
-          store_cols_bf16x2<16>(C, args.ldc, tl.row0 + c0 + mine, tl.rows - c0 - mine, col, args.nout, v);
+          const int mine = (int)rank * 16;
+          store_cols_bf16x2<16>(C, args.ldc, tl.row0 + j * 32 + mine, tl.rows - j * 32 - mine, col, args.nout, v);
         }
         if (!ok) break;
       }
