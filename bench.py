@@ -42,10 +42,14 @@ METRIC = "MoE-layer fwd tokens/s; expert GEMM TFLOP/s & HBM GB/s vs B200 peak"
 UNIT = "tokens/s"
 
 # DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu
-# capture, with the sha256 of the kernel source it was taken on; reported
-# only while the source is unchanged.
-TRAFFIC = {"kernel_sha": "dffd2674e8b13f24", "workload": "mixtral_bf16", "bytes": 2175553024,
-           "source": "profiles/gemm_tc_swiglu_mixtral_bf16.md"}
+# capture, with the sha256 of the kernel sources it was taken on; reported
+# only while those sources are unchanged.  The full DeepSeek-V3-shaped
+# prefill holds too much on the device for a multi-pass capture, so its
+# figure is the 32-expert case's DRAM bytes per algorithmic byte (1.0235),
+# applied to the full launch's algorithmic bytes: both are dominated by the
+# touched experts' weights, which every launch reads once.
+TRAFFIC = {"kernel_sha": "08252ee975d59be1", "workload": "dsv3_prefill_bf16", "per_algorithmic_byte": 1.0235,
+           "source": "profiles/gemm_swap_dsv3_prefill_shape.md (E = 32, N = 1024 case, scaled)"}
 
 
 def _peaks():
@@ -365,8 +369,9 @@ def run_native(args):
         # is reported beside it.
         peak, peak_sus = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
         sha = _kernel_sha()
-        traffic = TRAFFIC.get("bytes") if TRAFFIC.get("kernel_sha") == sha and \
-            TRAFFIC.get("workload") == args.workload and not args.set else None
+        traffic = round(TRAFFIC["per_algorithmic_byte"] * fb["gate_up_bytes"]) \
+            if TRAFFIC.get("kernel_sha") == sha and TRAFFIC.get("workload") == args.workload and not args.set \
+            and args.tiling == 0 else None
         kernel = ("grouped gate/up + SwiGLU GEMM (tcgen05)" +
                   (" incl. the folded shared expert" if fb["shared_folded"] else ""))
         # the dominant kernel is bound by whichever of its FLOPs and its bytes
