@@ -391,13 +391,19 @@ def test_folded_shared_expert_in_both_tilings(torch_cuda, gemm_tiling, mode):
 
 # ----------------------------------------------------------------- the forward pass as a CUDA graph
 
-@pytest.mark.parametrize("name", ["tiny_fp32", "dsv3_decode_bf16"])
+# the last case is the DeepSeek-V3 prefill's per-expert shape on 32 experts: the
+# swapped-operand GEMMs, the router on the tensor cores and the multi-kernel permute
+@pytest.mark.parametrize("name", ["tiny_fp32", "dsv3_decode_bf16", "dsv3_prefill_bf16:32x1024"])
 def test_layer_forward_replays_from_a_cuda_graph(torch_cuda, name):
     # moe_layer_forward enqueues work on one stream with no host synchronisation,
     # so a captured graph replays the identical computation
     torch = torch_cuda
     import sparse_mixture_experts_rmsnorm_b200 as moe
-    cfg = mi.CONFIGS[name]
+    base, _, size = name.partition(":")
+    cfg = mi.CONFIGS[base]
+    if size:
+        e, n = (int(v) for v in size.split("x"))
+        cfg = cfg.with_(n_experts=e, n_tokens=n)
     lc = lib_config(cfg)
     dev = mi.device_tensors(cfg)
     w = {n: dev[n] for n in ("norm_w", "w_router", "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down")
