@@ -71,6 +71,10 @@ constexpr int S_THREADS = 192;
 constexpr int S_CHUNK = 256;  // most rows of a group in one tile (the MMA's largest N)
 constexpr int S_RUN = 8;      // chunks that walk a group's weight tiles together
 constexpr int S_XMAPS = 16;   // row boxes of 8, 16, ..., 128 rows
+constexpr int S_TRING = 8;    // tile indices published ahead of the roles that read them
+// readers of each published tile index: the even CTA's MMA thread and 4 epilogue
+// warps, the odd CTA's producer and 4 epilogue warps
+constexpr int S_TRING_READERS = 10;
 
 struct SwapMaps {
   CUtensorMap w[2];            // routed weights: gate and up (SwiGLU) or down (w[1] = w[0]); 128-row boxes
@@ -92,7 +96,10 @@ struct SwapArgs {
   uint64_t wait_ns;
   int shared_group;  // group whose weights come from ws (-1: none)
   int shared_a;      // 1: that group's rows come from xs, from row 0
+  int* tile_counter; // zeroed before the launch: tiles claimed past the first one of each pair (nullptr: static)
 };
+
+enum { SITE_XFULL = 6, SITE_XEMPTY = 7, SITE_RING = 8 };  // wait sites of this kernel (error record word 3)
 
 struct SwapTile {
   int group, row0, rows, n, o;  // rows [row0, row0 + rows) of C; n = rows rounded up to 16; weight tile o
@@ -173,6 +180,10 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
   return ok != 0;
 }
 
+// One thread's bounded wait on a barrier that the other CTA of the pair may
+// arrive on (acquire at cluster scope).
+__device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity, const SwapArgs& a, volatile int* abort);
+
 // Warp-uniform bounded wait: lane 0 waits with the bound, the outcome goes to
 // every lane, and each lane then observes the completed phase itself (which
 // returns at once: the phase cannot move on without this warp).
@@ -206,6 +217,22 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const 
   return ok;
 }
 
+__device__ __forceinline__ bool ring_wait(uint64_t* bar, uint32_t parity, const SwapArgs& a, volatile int* abort) {
+  if (mbar_try_wait_cluster(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t polls = 1;; ++polls) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if ((polls & 63u) == 0u) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 >= a.wait_ns) {
+        record_error(a.hdr, MOE_ERR_DEVICE_TIMEOUT, KID_GEMM_TC, blockIdx.x, SITE_RING);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
 // Store ROWS accumulator columns of this lane's output column `col` (lane =
 // column; the block is rows row0 .. row0 + ROWS - 1 of C, the first `valid` of
 // them real).  Neighbouring lanes trade one value, so each lane stores two
@@ -230,7 +257,7 @@ __device__ __forceinline__ void store_cols_bf16x2(bf16* C, int ldc, int row0, in
   }
 }
 
-enum { SITE_XFULL = 6, SITE_XEMPTY = 7 };
+
 
 // silu(z) = z / (1 + e^-z) with the fast exp and divide intrinsics: about 1e-6
 // relative error in fp32, far below the bf16 rounding of the activation that
@@ -248,6 +275,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
   __shared__ __align__(8) uint64_t xfull_bar[4][2];      // SwiGLU: the partner's block for warp q, buffer b, arrived
   __shared__ __align__(8) uint64_t xempty_bar[4][2];     //         ... this CTA's block in the partner has been read
   __shared__ __align__(8) uint64_t drain_bar;
+  __shared__ __align__(8) uint64_t tr_full[S_TRING];   // a tile index is in tile_ring[j] (both CTAs)
+  __shared__ __align__(8) uint64_t tr_empty[S_TRING];  // every reader has taken it (even CTA)
+  __shared__ volatile int tile_ring[S_TRING];
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
   __shared__ int offs_sh[TC_MAX_GROUPS + 1];
@@ -279,6 +309,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
         mbar_init(&xfull_bar[q][b], 32);   // every lane of the partner warp
         mbar_init(&xempty_bar[q][b], 32);
       }
+    for (int j = 0; j < S_TRING; ++j) {
+      mbar_init(&tr_full[j], 1);
+      mbar_init(&tr_empty[j], S_TRING_READERS);
+    }
     mbar_init(&drain_bar, 1);
     fence_barrier_init();
   }
@@ -307,7 +341,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
       uint32_t phase = 0;
       long issued = 0;
       bool ok = true;
-      for (int t = first; t < total_tiles && ok; t += step) {
+      // Tiles: each pair starts with tile `first`; the even CTA's producer then
+      // claims the next unclaimed tile from the launch's counter and publishes
+      // every index (and finally one past the last tile) to the other roles of
+      // both CTAs through tile_ring.  The odd CTA's producer reads the ring too.
+      int rs = 0, t = first;
+      uint32_t rph = 0;
+      while (ok) {
+        if (leader) {
+          if (!mbar_wait_bounded(&tr_empty[rs], rph ^ 1u, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
+                                 SITE_RING)) {
+            ok = false;
+            break;
+          }
+          tile_ring[rs] = t;
+          asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(map_to_rank((const void*)&tile_ring[rs], 1)), "r"(t)
+                       : "memory");
+          mbar_arrive(&tr_full[rs]);
+          mbar_arrive_cluster(map_to_rank(&tr_full[rs], 1));
+        } else {
+          if (!ring_wait(&tr_full[rs], rph, args, &abort_flag)) {
+            ok = false;
+            break;
+          }
+          t = tile_ring[rs];
+          mbar_arrive_cluster(map_to_rank(&tr_empty[rs], 0));
+        }
+        if (++rs == S_TRING) {
+          rs = 0;
+          rph ^= 1u;
+        }
+        if (t >= total_tiles) break;
+        const int t_next = leader ? (args.tile_counter ? step + atomicAdd(args.tile_counter, 1) : t + step) : 0;
         const SwapTile tl = swap_decode(t, prefix_sh, offs_sh, G, args.n_o);
         const bool sh = tl.group == args.shared_group;  // the folded shared expert has its own weights
         const CUtensorMap* wm = sh ? &maps.ws[wsel] : &maps.w[wsel];
@@ -335,6 +400,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
             phase ^= 1u;
           }
         }
+        t = t_next;
       }
       // Drain (even CTA, which owns the full barriers): the last loads of
       // both CTAs have landed before exit.
@@ -359,7 +425,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
       int buf = 0;
       uint32_t bphase = 0;
       bool ok = true;
-      for (int t = first; t < total_tiles && ok; t += step) {
+      int rs = 0;
+      uint32_t rph = 0;
+      while (ok) {
+        if (!ring_wait(&tr_full[rs], rph, args, &abort_flag)) break;
+        const int t = tile_ring[rs];
+        mbar_arrive(&tr_empty[rs]);
+        if (++rs == S_TRING) {
+          rs = 0;
+          rph ^= 1u;
+        }
+        if (t >= total_tiles) break;
         const SwapTile tl = swap_decode(t, prefix_sh, offs_sh, G, args.n_o);
         const uint32_t idesc = tc_idesc(256, tl.n);
         const uint32_t b_kblk = (uint32_t)((tl.n >> 1) * TC_BK * 2);  // bytes of one k-block of this CTA's rows
@@ -414,7 +490,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
     uint32_t bphase = 0;
     uint32_t xi = 0;  // SwiGLU: 32-row blocks this warp has handled (buffer xi & 1, phase (xi >> 1) & 1)
     bool ok = true;
-    for (int t = first; t < total_tiles && ok; t += step) {
+    int rs = 0;
+    uint32_t rph = 0;
+    while (ok) {
+      if (!warp_wait(&tr_full[rs], rph, args, &abort_flag, SITE_RING, true)) break;
+      const int t = tile_ring[rs];
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_rank(&tr_empty[rs], 0));
+      if (++rs == S_TRING) {
+        rs = 0;
+        rph ^= 1u;
+      }
+      if (t >= total_tiles) break;
       const SwapTile tl = swap_decode(t, prefix_sh, offs_sh, G, args.n_o);
       if (!warp_wait(&tfull_bar[buf], bphase, args, &abort_flag, SITE_TMEM_FULL, false)) break;
       tc_fence_after();
@@ -630,6 +717,12 @@ moe_status launch_gemm_swap(int epi, const void* a, const void* b, const void* b
   args.wait_ns = wait_limit_ns();
   args.shared_group = (sb != nullptr && offsets) ? groups - 1 : -1;
   args.shared_a = shared_a ? 1 : 0;
+  // the tile counter lives in the workspace header (word 32), zeroed for every launch
+  args.tile_counter = nullptr;
+  if (hdr != nullptr) {
+    args.tile_counter = hdr + 32;
+    if (cudaMemsetAsync(args.tile_counter, 0, sizeof(int), s) != cudaSuccess) return MOE_ERR_CUDA;
+  }
   // upper bound on the tiles; the exact count lives on the device
   const int64_t chunks = (int64_t)(max_rows + moe::S_CHUNK - 1) / moe::S_CHUNK + args.groups;
   const int64_t bound = chunks * args.n_o;
