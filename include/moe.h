@@ -114,8 +114,10 @@ const char* moe_version(void);
 
 /* Bytes of device workspace that moe_layer_forward needs for this config,
  * and that is also enough for every staged call below with the same config;
- * 0 if the config is invalid.  The workspace holds a 256-byte header (device
- * error word), xn, the routing buffers that moe_routing leaves NULL, router
+ * 0 if the config is invalid.  The workspace holds a 256-byte header (the
+ * device error word, and the tile counter of the swapped-operand expert GEMMs,
+ * which each of their launches zeroes first), xn, the routing buffers that
+ * moe_routing leaves NULL, router
  * logits, permutation histograms, the expert-sorted rows x_perm [R][d],
  * activations [max(R*H, N*Hs)] and expert outputs y_perm [R][d], y_shared
  * [N][d], where R = N*k, or min(N*k, E*cap) with a capacity.  When the
