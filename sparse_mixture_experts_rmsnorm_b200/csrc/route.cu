@@ -26,7 +26,7 @@ namespace moe {
 // row is staged in shared memory in its own dtype; when `logits` is given, the
 // block's warps then take the router dot products of the rounded xn row
 // with experts [e0, e0 + epb) (e0 = blockIdx.y * epb), one expert per warp
-// at a time, fp32 FMA per lane and a warp tree sum.  Blocks with
+// at a time, fp32 FMA per lane (dot_accum) and a warp tree sum.  Blocks with
 // blockIdx.y == 0 write xn.
 // ---------------------------------------------------------------------------
 template <typename T, int V>
@@ -53,6 +53,43 @@ template <typename T, int V>
 __device__ __forceinline__ void st_vec(T* p, const Vec<T, V>& x) {
   if (V * sizeof(T) == 16) *reinterpret_cast<uint4*>(p) = *reinterpret_cast<const uint4*>(&x);
   else p[0] = x.v[0];
+}
+
+// s += x[j] * w[j] for j = 0 .. V-1 in order, each an fp32 FMA with one
+// rounding.  A bf16 value widens to fp32 exactly, so the bf16 form below (the
+// sm_100 FMA that takes bf16 sources and an fp32 addend and result) gives the
+// same bits as widening both operands first, without the conversions that
+// otherwise take most of the router's issue slots.
+template <typename T, int V>
+__device__ __forceinline__ float dot_accum(const T* x, const T* w, float s) {
+  float xf[V], wf[V];
+  vec_to_f32(ld_vec<T, V>(x), xf);
+  vec_to_f32(ld_vec<T, V>(w), wf);
+#pragma unroll
+  for (int j = 0; j < V; ++j) s = __fmaf_rn(xf[j], wf[j], s);
+  return s;
+}
+
+__device__ __forceinline__ float fma_bf16x2(uint32_t a, uint32_t b, float c) {
+  asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+      "mov.b32 {al, ah}, %1;\n\t"
+      "mov.b32 {bl, bh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, al, bl, %0;\n\t"
+      "fma.rn.f32.bf16 %0, ah, bh, %0;\n\t}"
+      : "+f"(c)
+      : "r"(a), "r"(b));
+  return c;
+}
+
+template <>
+__device__ __forceinline__ float dot_accum<bf16, 8>(const bf16* x, const bf16* w, float s) {
+  const uint4 a = *reinterpret_cast<const uint4*>(x);
+  const uint4 b = *reinterpret_cast<const uint4*>(w);
+  s = fma_bf16x2(a.x, b.x, s);
+  s = fma_bf16x2(a.y, b.y, s);
+  s = fma_bf16x2(a.z, b.z, s);
+  s = fma_bf16x2(a.w, b.w, s);
+  return s;
 }
 
 template <typename T, int V>
@@ -106,13 +143,7 @@ __global__ void __launch_bounds__(256) rmsnorm_router_kernel(const T* __restrict
       for (int e = e0 + warp_id(); e < e1; e += warps) {
         const T* wr = w_router + (size_t)e * d;
         float s = 0.f;
-        for (int i = lane_id() * V; i < d; i += 32 * V) {
-          float xf[V], wf[V];
-          vec_to_f32(ld_vec<T, V>(row + i), xf);
-          vec_to_f32(ld_vec<T, V>(wr + i), wf);
-#pragma unroll
-          for (int j = 0; j < V; ++j) s = __fmaf_rn(xf[j], wf[j], s);
-        }
+        for (int i = lane_id() * V; i < d; i += 32 * V) s = dot_accum<T, V>(row + i, wr + i, s);
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
         if (lane_id() == 0) logits[(size_t)t * E + e] = s;
