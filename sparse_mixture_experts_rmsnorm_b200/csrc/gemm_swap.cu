@@ -345,34 +345,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
       // claims the next unclaimed tile from the launch's counter and publishes
       // every index (and finally one past the last tile) to the other roles of
       // both CTAs through tile_ring.  The odd CTA's producer reads the ring too.
-      int rs = 0, t = first;
+      // A tile's successor is published right after the tile's first stage is
+      // issued, so both producers already hold it when the tile's last stage
+      // is out, and the claim behind it was made a whole tile earlier (the
+      // atomic's round trip and the cross-CTA publish stay off the boundary).
+      int rs = 0;
       uint32_t rph = 0;
-      while (ok) {
-        if (leader) {
-          if (!mbar_wait_bounded(&tr_empty[rs], rph ^ 1u, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
-                                 SITE_RING)) {
-            ok = false;
-            break;
-          }
-          tile_ring[rs] = t;
-          asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(map_to_rank((const void*)&tile_ring[rs], 1)), "r"(t)
-                       : "memory");
-          mbar_arrive(&tr_full[rs]);
-          mbar_arrive_cluster(map_to_rank(&tr_full[rs], 1));
-        } else {
-          if (!ring_wait(&tr_full[rs], rph, args, &abort_flag)) {
-            ok = false;
-            break;
-          }
-          t = tile_ring[rs];
-          mbar_arrive_cluster(map_to_rank(&tr_empty[rs], 0));
-        }
+      auto publish = [&](int v) -> bool {
+        if (!mbar_wait_bounded(&tr_empty[rs], rph ^ 1u, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
+                               SITE_RING))
+          return false;
+        tile_ring[rs] = v;
+        asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(map_to_rank((const void*)&tile_ring[rs], 1)), "r"(v)
+                     : "memory");
+        mbar_arrive(&tr_full[rs]);
+        mbar_arrive_cluster(map_to_rank(&tr_full[rs], 1));
         if (++rs == S_TRING) {
           rs = 0;
           rph ^= 1u;
         }
-        if (t >= total_tiles) break;
-        const int t_next = leader ? (args.tile_counter ? step + atomicAdd(args.tile_counter, 1) : t + step) : 0;
+        return true;
+      };
+      auto take = [&](int& v) -> bool {
+        if (!ring_wait(&tr_full[rs], rph, args, &abort_flag)) return false;
+        v = tile_ring[rs];
+        mbar_arrive_cluster(map_to_rank(&tr_empty[rs], 0));
+        if (++rs == S_TRING) {
+          rs = 0;
+          rph ^= 1u;
+        }
+        return true;
+      };
+      // the tile after `prev` in the launch's order: the counter's next, else the pair's static successor
+      auto claim = [&](int prev) -> int { return args.tile_counter ? step + atomicAdd(args.tile_counter, 1) : prev + step; };
+      int t = first;
+      int pending = 0;  // even CTA: the claimed successor of the next tile
+      if (leader) {
+        ok = publish(t);
+        if (ok && t < total_tiles) pending = claim(t);
+      } else {
+        ok = take(t);
+      }
+      while (ok && t < total_tiles) {
         const SwapTile tl = swap_decode(t, prefix_sh, offs_sh, G, args.n_o);
         const bool sh = tl.group == args.shared_group;  // the folded shared expert has its own weights
         const CUtensorMap* wm = sh ? &maps.ws[wsel] : &maps.w[wsel];
@@ -383,6 +397,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
         const int w_base = sh ? 0 : tl.group * args.nout;
         const int w_row = EPI == moe_host::EPI_SWIGLU ? w_base + tl.o * 128 : w_base + tl.o * 256 + (int)rank * 128;
         const uint32_t tx = 2u * (uint32_t)(S_A_BYTES + S_KB * half * TC_BK * 2);
+        int next = 0;
+        bool sent = !leader;  // the even CTA still owes the ring this tile's successor
         for (int ks = 0; ks < n_stage_tiles; ++ks) {
           if (!mbar_wait_bounded(&empty_bar[stage], phase ^ 1u, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
                                  SITE_EMPTY)) {
@@ -399,8 +415,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
             stage = 0;
             phase ^= 1u;
           }
+          if (!sent) {
+            sent = true;
+            next = pending;
+            if (!publish(next)) {
+              ok = false;
+              break;
+            }
+            if (next < total_tiles) pending = claim(next);
+          }
         }
-        t = t_next;
+        if (!ok) break;
+        if (leader) {
+          t = next;
+        } else if (!take(t)) {
+          break;
+        }
       }
       // Drain (even CTA, which owns the full barriers): the last loads of
       // both CTAs have landed before exit.
@@ -666,7 +696,7 @@ static moe_status launch_swap_t(const moe::SwapMaps& maps, const moe::SwapArgs& 
 }
 
 bool swap_supported(int epi, int nout, int k, int ldc) {
-  return epi != EPI_F32 && k % moe::TC_BK == 0 && nout % 8 == 0 && ldc % 8 == 0;
+  return epi != EPI_F32 && k >= moe::TC_BK && k % moe::TC_BK == 0 && nout % 8 == 0 && ldc % 8 == 0;
 }
 
 moe_status launch_gemm_swap(int epi, const void* a, const void* b, const void* b2, const int32_t* offsets,

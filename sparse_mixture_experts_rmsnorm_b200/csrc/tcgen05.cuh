@@ -330,7 +330,7 @@ moe_status launch_gemm_tc2(int epi, const CUtensorMap& ma, const CUtensorMap& mb
 
 // The swapped-operand SM-pair kernel (gemm_swap.cu), same arguments as
 // launch_gemm_tc; SwiGLU and plain-store epilogues, bf16 only, for the shapes
-// swap_supported accepts (K a multiple of 64, nout and ldc multiples of 8).
+// swap_supported accepts (K a positive multiple of 64, nout and ldc multiples of 8).
 bool swap_supported(int epi, int nout, int k, int ldc);
 moe_status launch_gemm_swap(int epi, const void* a, const void* b, const void* b2, const int32_t* offsets,
                             int groups, int max_rows, int nout, int k, void* c, int ldc, int32_t* hdr,
