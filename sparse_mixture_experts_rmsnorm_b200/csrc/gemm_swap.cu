@@ -306,8 +306,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
     }
     for (int q = 0; q < 4; ++q)
       for (int b = 0; b < 2; ++b) {
-        mbar_init(&xfull_bar[q][b], 32);   // every lane of the partner warp
-        mbar_init(&xempty_bar[q][b], 32);
+        mbar_init(&xfull_bar[q][b], 1);   // lane 0 of the partner warp (plus its st.async bytes)
+        mbar_init(&xempty_bar[q][b], 1);
       }
     for (int j = 0; j < S_TRING; ++j) {
       mbar_init(&tr_full[j], 1);
@@ -356,10 +356,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
                                SITE_RING))
           return false;
         tile_ring[rs] = v;
-        asm volatile("st.shared::cluster.b32 [%0], %1;" ::"r"(map_to_rank((const void*)&tile_ring[rs], 1)), "r"(v)
-                     : "memory");
         mbar_arrive(&tr_full[rs]);
-        mbar_arrive_cluster(map_to_rank(&tr_full[rs], 1));
+        // the odd CTA's copy: the word and its barrier's completion travel together
+        const uint32_t peer_full = map_to_rank(&tr_full[rs], 1);
+        mbar_arrive_expect_tx_cluster(peer_full, 4);
+        st_async_b32(map_to_rank((const void*)&tile_ring[rs], 1), (uint32_t)v, peer_full);
         if (++rs == S_TRING) {
           rs = 0;
           rph ^= 1u;
@@ -369,7 +370,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
       auto take = [&](int& v) -> bool {
         if (!ring_wait(&tr_full[rs], rph, args, &abort_flag)) return false;
         v = tile_ring[rs];
-        mbar_arrive_cluster(map_to_rank(&tr_empty[rs], 0));
+        mbar_arrive_cluster_relaxed(map_to_rank(&tr_empty[rs], 0) + depend_zero((uint32_t)v));
         if (++rs == S_TRING) {
           rs = 0;
           rph ^= 1u;
@@ -525,8 +526,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
     while (ok) {
       if (!warp_wait(&tr_full[rs], rph, args, &abort_flag, SITE_RING, true)) break;
       const int t = tile_ring[rs];
+      const uint32_t z = depend_zero((uint32_t)t);  // every lane's read has returned ...
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(map_to_rank(&tr_empty[rs], 0));
+      if (lane == 0) mbar_arrive_cluster_relaxed(map_to_rank(&tr_empty[rs], 0) + z);  // ... before the slot is freed
       if (++rs == S_TRING) {
         rs = 0;
         rph ^= 1u;
@@ -571,13 +573,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
             snd[i] = leader ? a[16 + i] : a[i];
             own[i] = leader ? a[i] : a[16 + i];
           }
+          // the values and the partner's barrier completion travel together (st.async)
           const uint32_t dst = map_to_rank_addr(xrow + (uint32_t)(b * S_XCH_BYTES), peer);
+          const uint32_t peer_full = map_to_rank(&xfull_bar[quarter][b], peer);
+          if (lane == 0) mbar_arrive_expect_tx_cluster(peer_full, 32u * 16u * 4u);
 #pragma unroll
           for (int i = 0; i < 16; i += 4)
-            asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst + (uint32_t)(i * 4)),
-                         "r"(snd[i]), "r"(snd[i + 1]), "r"(snd[i + 2]), "r"(snd[i + 3])
-                         : "memory");
-          mbar_arrive_cluster(map_to_rank(&xfull_bar[quarter][b], peer));
+            st_async_v4(dst + (uint32_t)(i * 4), snd[i], snd[i + 1], snd[i + 2], snd[i + 3], peer_full);
           return true;
         };
         if (nblk > 0 && !send_block(0, xi)) {
@@ -614,7 +616,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(S_THREADS, 1)
               v[i + e] = __fmul_rn(silu_fast(g), up);
             }
           }
-          mbar_arrive_cluster(map_to_rank(&xempty_bar[quarter][b], peer));
+          // every lane's reads of the buffer have returned (v depends on all four loads) before
+          // lane 0 lets the partner overwrite it
+          const uint32_t z = depend_zero(__float_as_uint(v[3]) ^ __float_as_uint(v[7]) ^ __float_as_uint(v[11]) ^
+                                         __float_as_uint(v[15]));
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster_relaxed(map_to_rank(&xempty_bar[quarter][b], peer) + z);
           const int mine = (int)rank * 16;
           store_cols_bf16x2<16>(C, args.ldc, tl.row0 + j * 32 + mine, tl.rows - j * 32 - mine, col, args.nout, v);
         }

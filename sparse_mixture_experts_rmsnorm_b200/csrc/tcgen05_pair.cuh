@@ -72,5 +72,43 @@ __device__ __forceinline__ void tc2_commit_own(uint64_t* bar) {
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
 }
+// The same arrival without the cluster-scope release, so the thread does not
+// wait for its earlier memory operations to be performed at cluster scope.
+// For a barrier that guards a slot this thread has just READ: pass the read
+// value through depend_zero into the address, so the arrive cannot issue
+// before the load has returned (the slot may be rewritten only after it).
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t bar_cluster) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(bar_cluster) : "memory");
+}
+// 0, computed from v: an instruction that reads v, so its result is ready only
+// once v's load has returned.
+__device__ __forceinline__ uint32_t depend_zero(uint32_t v) {
+  uint32_t z;
+  asm volatile("and.b32 %0, %1, 0;" : "=r"(z) : "r"(v));
+  return z;
+}
+// 16 bytes into the other CTA's shared memory, counted on its barrier like st_async_b32.
+__device__ __forceinline__ void st_async_v4(uint32_t dst_cluster, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                            uint32_t bar_cluster) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   dst_cluster),
+               "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar_cluster)
+               : "memory");
+}
+// Arrive on a barrier of the pair and add `bytes` to the transfer it awaits
+// (data that st.async below delivers); no release.
+__device__ __forceinline__ void mbar_arrive_expect_tx_cluster(uint32_t bar_cluster, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.relaxed.cluster.shared::cluster.b64 _, [%0], %1;" ::"r"(bar_cluster),
+               "r"(bytes)
+               : "memory");
+}
+// Store one word into the other CTA's shared memory; its barrier counts the 4
+// bytes as transferred once the word is written, so a reader that sees the
+// barrier's phase complete (acquire at cluster scope) sees the word.
+__device__ __forceinline__ void st_async_b32(uint32_t dst_cluster, uint32_t v, uint32_t bar_cluster) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(dst_cluster), "r"(v),
+               "r"(bar_cluster)
+               : "memory");
+}
 
 }  // namespace moe
