@@ -264,13 +264,13 @@ moe_status moe_set_wait_timeout_ns(int64_t ns);
 /* Tile shape of the bf16 grouped expert GEMMs for launches after this call
  * (process-wide): 0 = choose per launch (the default: SM-pair tiles with the
  * operands swapped -- 256 weight rows on M, up to 256 of a group's rows on
- * N, padded to 16 -- for the down projection when the groups average at
- * least 64 rows and H % 64 == 0, and for the gate/up projection when 16 or
- * more groups average 64 to 511 rows and d % 64 == 0; single-SM 128-row
- * tiles for the other gate/up launches; for the other down projections of
- * groups averaging at least 512 rows, single-SM or SM-pair 256-row tiles
- * picked on the device from the group sizes; the router takes SM pairs from
- * 512 tokens), 1 = single-SM tiles, 2 = SM-pair
+ * N, padded to 16 -- for every gate/up projection with d % 64 == 0, and for
+ * the down projection when the groups average at least 64 rows and
+ * H % 64 == 0; single-SM 128-row tiles (64-row for small groups) for the
+ * other gate/up launches and the other down projections of smaller groups;
+ * for the other down projections of groups averaging at least 512 rows,
+ * single-SM or SM-pair 256-row tiles picked on the device from the group
+ * sizes; the router takes SM pairs from 512 tokens), 1 = single-SM tiles, 2 = SM-pair
  * tiles, 3 = swapped-operand SM-pair tiles for both expert GEMMs where the
  * shape allows (K % 64 == 0; the router keeps the automatic choice).  Results are
  * the same up to floating-point summation order; this is a performance

@@ -418,17 +418,18 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
   const int forced = tc_pairing();
   // Operands swapped on SM pairs (gemm_swap.cu): weight rows on M, the
   // group's rows on N in chunks of at most 256 padded to 16 (K a multiple of
-  // 64).  Measured on B200 (same box, one run each):
-  //  - the down projection of every prefill-sized workload (groups averaging
-  //    >= 64 rows) is fastest this way: DeepSeek-V3-shaped 2.25 against
-  //    2.47 ms, Mixtral-shaped 0.67 against 0.74 ms (and 0.88 with SM pairs),
-  //    load-imbalance 0.53 against 0.56 ms;
-  //  - the SwiGLU projection only where there are many groups of a few
-  //    hundred rows: DeepSeek-V3-shaped 4.54 against 4.66 ms, but
-  //    Mixtral-shaped (8 groups of 1024) 2.05 against 1.67 ms;
-  //  - decode (2 rows a group) keeps the M = 64 tiles.
-  const bool swap_auto = forced == 0 && offsets != nullptr && rows_per_group >= 64 &&
-                         (epi == EPI_STORE || (epi == EPI_SWIGLU && groups >= 16 && rows_per_group < 512));
+  // 64).  Measured on B200 (same box, interleaved processes):
+  //  - the SwiGLU projection is fastest this way on every grouped workload:
+  //    DeepSeek-V3-shaped prefill 4.54 against 4.66 ms, Mixtral-shaped
+  //    (8 groups of 1024) 1.58-1.61 against 1.70-1.71 ms, load-imbalance
+  //    1.09-1.10 against 1.18-1.19 ms, decode (2 rows a group) 1.94 against
+  //    2.00 ms;
+  //  - the down projection when groups average >= 64 rows: DeepSeek-V3-shaped
+  //    2.25 against 2.47 ms, Mixtral-shaped 0.67 against 0.74 ms (and 0.88
+  //    with SM pairs), load-imbalance 0.53 against 0.56 ms; decode keeps the
+  //    M = 64 tiles (0.97 ms either way).
+  const bool swap_auto = forced == 0 && offsets != nullptr &&
+                         (epi == EPI_SWIGLU || (epi == EPI_STORE && rows_per_group >= 64));
   if ((forced == 3 || swap_auto) && swap_supported(epi, nout, k, ldc))
     return launch_gemm_swap(epi, a, b, b2, offsets, groups, max_rows, nout, k, c, ldc, hdr, s, sb, sb2, sa, sa_rows);
   const int mode = forced == 3 ? 0 : forced;  // the router's fp32 logits: the automatic choice
