@@ -45,10 +45,10 @@ UNIT = "tokens/s"
 # capture, with the sha256 of the kernel sources it was taken on; reported
 # only while those sources are unchanged.  The full DeepSeek-V3-shaped
 # prefill holds too much on the device for a multi-pass capture, so its
-# figure is the 32-expert case's DRAM bytes per algorithmic byte (1.0172),
+# figure is the 32-expert case's DRAM bytes per algorithmic byte (1.0211),
 # applied to the full launch's algorithmic bytes: both are dominated by the
 # touched experts' weights, which every launch reads once.
-TRAFFIC = {"kernel_sha": "383314e89716039c", "workload": "dsv3_prefill_bf16", "per_algorithmic_byte": 1.0172,
+TRAFFIC = {"kernel_sha": "f929f29a69c46967", "workload": "dsv3_prefill_bf16", "per_algorithmic_byte": 1.0211,
            "source": "profiles/gemm_swap_dsv3_prefill_shape.md (E = 32, N = 1024 case, scaled)"}
 
 
