@@ -67,15 +67,16 @@ __global__ void __launch_bounds__(kPermWarps * 32) chunk_hist_kernel(const int32
 }
 
 // One block of 1024 threads.
-//   1. Each warp takes whole experts: the exclusive scan of hist[e][*] over
-//      the chunks, in place, gives every chunk the rank of its first slot of
-//      expert e; the row total is count_e (also written to `counts` when
-//      given).  The warp loads 32 * kScanPer chunk counts with coalesced,
-//      independent loads, scans them as kScanPer warp scans in registers and
-//      stores them back coalesced: one memory round trip per 32 * kScanPer
-//      chunks.
+//   1. Each warp takes whole experts, kScanExp at a time: the exclusive scan
+//      of hist[e][*] over the chunks, in place, gives every chunk the rank of
+//      its first slot of expert e; the row total is count_e (also written to
+//      `counts` when given).  The warp loads kScanExp rows of 32 * kScanPer
+//      chunk counts with coalesced, independent loads, scans them as warp
+//      scans in registers and stores them back coalesced: one memory round
+//      trip per kScanExp experts and 32 * kScanPer chunks.
 //   2. kept_e = min(count_e, cap); offsets = exclusive scan of kept (E+1).
 constexpr int kScanPer = 8;
+constexpr int kScanExp = 4;
 
 __global__ void __launch_bounds__(1024) hist_scan_kernel(int32_t* __restrict__ hist, int E, int nchunks, int cap,
                                                          int32_t* __restrict__ offsets,
@@ -84,37 +85,54 @@ __global__ void __launch_bounds__(1024) hist_scan_kernel(int32_t* __restrict__ h
   __shared__ int32_t kept_sh[1024];
   __shared__ int32_t warp_sum[32];
   const int lane = lane_id(), warp = warp_id();
-  for (int e = warp; e < E; e += 32) {
-    int32_t* row = hist + (int64_t)e * nchunks;
-    int32_t carry = 0;
+  for (int e0 = warp; e0 < E; e0 += 32 * kScanExp) {
+    int32_t carry[kScanExp];
+#pragma unroll
+    for (int b = 0; b < kScanExp; ++b) carry[b] = 0;
     for (int c0 = 0; c0 < nchunks; c0 += 32 * kScanPer) {
-      int32_t v[kScanPer];
+      int32_t v[kScanExp][kScanPer];
 #pragma unroll
-      for (int i = 0; i < kScanPer; ++i) {
-        const int c = c0 + 32 * i + lane;
-        v[i] = (c < nchunks) ? row[c] : 0;
-      }
+      for (int b = 0; b < kScanExp; ++b) {
+        const int e = e0 + 32 * b;
 #pragma unroll
-      for (int i = 0; i < kScanPer; ++i) {
-        if (c0 + 32 * i >= nchunks) break;  // uniform across the warp
-        int32_t x = v[i];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          int32_t y = __shfl_up_sync(0xffffffffu, x, o);
-          if (lane >= o) x += y;
+        for (int i = 0; i < kScanPer; ++i) {
+          const int c = c0 + 32 * i + lane;
+          v[b][i] = (e < E && c < nchunks) ? hist[(int64_t)e * nchunks + c] : 0;
         }
-        v[i] = carry + x - v[i];
-        carry += __shfl_sync(0xffffffffu, x, 31);
       }
 #pragma unroll
-      for (int i = 0; i < kScanPer; ++i) {
-        const int c = c0 + 32 * i + lane;
-        if (c < nchunks) row[c] = v[i];
+      for (int b = 0; b < kScanExp; ++b) {
+#pragma unroll
+        for (int i = 0; i < kScanPer; ++i) {
+          int32_t x = v[b][i];
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            int32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+          }
+          v[b][i] = carry[b] + x - v[b][i];
+          carry[b] += __shfl_sync(0xffffffffu, x, 31);
+        }
+      }
+#pragma unroll
+      for (int b = 0; b < kScanExp; ++b) {
+        const int e = e0 + 32 * b;
+        if (e >= E) continue;  // uniform across the warp
+#pragma unroll
+        for (int i = 0; i < kScanPer; ++i) {
+          const int c = c0 + 32 * i + lane;
+          if (c < nchunks) hist[(int64_t)e * nchunks + c] = v[b][i];
+        }
       }
     }
     if (lane == 0) {
-      kept_sh[e] = (cap >= 0 && carry > cap) ? cap : carry;
-      if (counts != nullptr) counts[e] = carry;
+#pragma unroll
+      for (int b = 0; b < kScanExp; ++b) {
+        const int e = e0 + 32 * b;
+        if (e >= E) continue;
+        kept_sh[e] = (cap >= 0 && carry[b] > cap) ? cap : carry[b];
+        if (counts != nullptr) counts[e] = carry[b];
+      }
     }
   }
   __syncthreads();

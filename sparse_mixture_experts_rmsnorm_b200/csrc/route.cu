@@ -156,11 +156,20 @@ __global__ void __launch_bounds__(256) rmsnorm_router_kernel(const T* __restrict
 // ---------------------------------------------------------------------------
 // a3. One warp per token.  Lane l holds experts l, l + 32, ... (EPL of them).
 //   score = softmax(logits) in fp32; key = fl32(score + bias);
-//   k rounds of a warp arg-max on key (equal keys: lower expert wins);
+//   k rounds of a warp arg-max on key (equal keys: lower expert wins), each a
+//   lane-local scan and two warp reductions (largest key, then lowest expert
+//   holding it);
 //   gate_j = score_j / sum of the chosen scores.
 // counts: per-block shared histogram, added to the global one at the end
 // (skipped when counts is null).
 // ---------------------------------------------------------------------------
+// Unsigned image of a float that orders as the float does (-0 taken as +0,
+// so equal keys map to equal images).
+__device__ __forceinline__ uint32_t ordered_bits(float x) {
+  const uint32_t u = __float_as_uint(__fadd_rn(x, 0.0f));
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 template <int EPL>
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits,
                                                    const float* __restrict__ bias, float* __restrict__ scores,
@@ -207,36 +216,34 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     float my_score = 0.f;  // lane j < k keeps the score of the j-th choice
     int my_idx = 0;
     for (int j = 0; j < k; ++j) {
+      // this lane's best free expert (strict >: the lowest i, i.e. the lowest
+      // expert, among equal keys) ...
       float bk = -INFINITY;
-      int be = 0x7fffffff;
-      float bs = 0.f;
+      int bi = -1;
 #pragma unroll
       for (int i = 0; i < EPL; ++i) {
-        int e = lane + 32 * i;
-        bool free_ = !((taken >> i) & 1u) && e < E;
-        if (free_ && (key[i] > bk || (key[i] == bk && e < be))) {
+        const bool free_ = !((taken >> i) & 1u) && lane + 32 * i < E;
+        if (free_ && (bi < 0 || key[i] > bk)) {
           bk = key[i];
-          be = e;
-          bs = v[i];
+          bi = i;
         }
       }
+      // ... then the warp's largest key, and the lowest expert holding it
+      const uint32_t mk = bi >= 0 ? ordered_bits(bk) : 0u;
+      const uint32_t kmax = __reduce_max_sync(0xffffffffu, mk);
+      const uint32_t be = __reduce_min_sync(0xffffffffu, (bi >= 0 && mk == kmax) ? (uint32_t)(lane + 32 * bi)
+                                                                                   : 0xffffffffu);
+      const int wi = (int)(be >> 5);
+      float mine = v[0];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-        int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        float os = __shfl_xor_sync(0xffffffffu, bs, o);
-        if (ok > bk || (ok == bk && oe < be)) {
-          bk = ok;
-          be = oe;
-          bs = os;
-        }
-      }
-      // every lane now holds the winner (be, bs)
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      for (int i = 1; i < EPL; ++i)
+        if (wi == i) mine = v[i];
+      const float bs = __shfl_sync(0xffffffffu, mine, (int)(be & 31u));  // the winner's score
+      if ((int)(be & 31u) == lane) taken |= 1u << wi;
       chosen_sum = __fadd_rn(chosen_sum, bs);
       if (lane == j) {
         my_score = bs;
-        my_idx = be;
+        my_idx = (int)be;
       }
     }
     if (lane < k) {
