@@ -43,6 +43,7 @@ constexpr size_t kHeaderBytes = 256;
 enum KernelId : int32_t {
   KID_GEMM_TC = 1,
   KID_SELFTEST = 2,
+  KID_SCATTER = 3,
 };
 
 __device__ __forceinline__ void record_error(int32_t* hdr, int32_t status, int32_t kernel, int32_t block,

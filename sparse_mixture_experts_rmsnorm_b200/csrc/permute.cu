@@ -322,6 +322,89 @@ __global__ void __launch_bounds__(128) scatter_rows_kernel(const V* __restrict__
   }
 }
 
+// The same scatter with bulk copies (the copy engine moves whole rows, the
+// SM only issues them).  One warp per block; lane 0 keeps kBulkRing rows of
+// the block's tokens (t = blockIdx.x, + gridDim.x, ...) in flight: each row
+// arrives in shared memory by one bulk load completing on that buffer's
+// mbarrier, then leaves by one bulk store per kept slot (and the shared
+// expert's row), committed as one bulk group.  A buffer is reloaded once the
+// group that read it has finished reading (wait_group.read).  Lane j < nd
+// holds destination j of the next token, loaded a token ahead.  Rows must be
+// 16-byte aligned and a multiple of 16 bytes.
+constexpr int kBulkRing = 4;
+
+__global__ void __launch_bounds__(32) scatter_rows_bulk_kernel(const uint8_t* __restrict__ xn,
+                                                               const int32_t* __restrict__ slot_row,
+                                                               const int32_t* __restrict__ offsets, int E, int n,
+                                                               int k, uint8_t* __restrict__ x_perm,
+                                                               uint32_t row_bytes, int shared_rows,
+                                                               int32_t* __restrict__ hdr, uint64_t wait_ns) {
+  extern __shared__ __align__(128) uint8_t rows[];
+  __shared__ __align__(8) uint64_t full[kBulkRing];
+  const int lane = lane_id();
+  const int routed = offsets[E];
+  const int nd = k + (shared_rows > 0 ? 1 : 0);
+  const int64_t count = (n - (int64_t)blockIdx.x + gridDim.x - 1) / gridDim.x;  // this block's tokens
+  if (lane == 0) {
+    for (int b = 0; b < kBulkRing; ++b) mbar_init(&full[b], 1);
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the copy engine sees the initialised barriers
+  }
+  __syncwarp();
+  auto token = [&](int64_t i) { return (int64_t)blockIdx.x + i * gridDim.x; };
+  auto dst_of = [&](int64_t i) -> int {  // this lane's destination of the block's i-th token, or -1
+    if (i >= count || lane >= nd) return -1;
+    const int64_t t = token(i);
+    if (lane < k) return slot_row[t * k + lane];
+    return t < shared_rows ? routed + (int)t : -1;
+  };
+  auto load = [&](int64_t i) {
+    if (lane != 0 || i >= count) return;
+    const int b = (int)(i % kBulkRing);
+    mbar_arrive_expect_tx(&full[b], row_bytes);
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(rows + (size_t)b * row_bytes)),
+        "l"(xn + token(i) * row_bytes), "r"(row_bytes), "r"(smem_u32(&full[b]))
+        : "memory");
+  };
+  for (int64_t i = 0; i < kBulkRing - 1; ++i) load(i);
+  int d_cur = dst_of(0);
+  int64_t i = 0;
+  for (; i < count; ++i) {
+    const int d_next = dst_of(i + 1);  // in flight while this token is handled
+    const int b = (int)(i % kBulkRing);
+    bool landed = true;
+    if (lane == 0)
+      landed = mbar_wait_bounded(&full[b], (uint32_t)((i / kBulkRing) & 1), wait_ns, nullptr, hdr, KID_SCATTER, 1);
+    if (!__shfl_sync(0xffffffffu, landed, 0)) break;
+    const uint32_t src = smem_u32(rows + (size_t)b * row_bytes);
+    for (int j = 0; j < nd; ++j) {
+      const int r = __shfl_sync(0xffffffffu, d_cur, j);
+      if (lane == 0 && r >= 0)
+        asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(x_perm +
+                                                                                        (size_t)r * row_bytes),
+                     "r"(src), "r"(row_bytes)
+                     : "memory");
+    }
+    if (lane == 0) {
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      // the previous token's stores have read their buffer, which the next load reuses
+      asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+    }
+    __syncwarp();
+    load(i + kBulkRing - 1);
+    d_cur = d_next;
+  }
+  if (lane == 0) {
+    // After a failed wait, the loads still in flight land before the block
+    // exits (each wait bounded; the first failure is already recorded).
+    for (int64_t j = i; j < i + kBulkRing - 1 && j < count; ++j)
+      mbar_wait_bounded(&full[j % kBulkRing], (uint32_t)((j / kBulkRing) & 1), wait_ns, nullptr, nullptr,
+                        KID_SCATTER, 1);
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+  }
+}
+
 }  // namespace moe
 
 namespace moe_host {
@@ -363,11 +446,26 @@ moe_status launch_permute(const int32_t* topk_idx, int n, int k, int e, int cap,
 }
 
 moe_status launch_gather(int dtype, const void* xn, const int32_t* slot_row, const int32_t* offsets, int e, int n,
-                         int k, void* x_perm, int d, cudaStream_t s, int shared_rows) {
+                         int k, void* x_perm, int d, cudaStream_t s, int shared_rows, int32_t* hdr) {
   if (n == 0) return MOE_OK;
   if (k > 32) return MOE_ERR_UNSUPPORTED;
   const size_t row_bytes = (size_t)d * (dtype == MOE_BF16 ? 2 : 4);
   const uintptr_t addr = (uintptr_t)xn | (uintptr_t)x_perm;
+  // Bulk copies once there are enough tokens to keep every SM's copies busy
+  // (the block-per-token kernel below splits rows over blocks for fewer).
+  const size_t bulk_smem = moe::kBulkRing * row_bytes;
+  if (row_bytes % 16 == 0 && addr % 16 == 0 && n >= 2 * sm_count() && bulk_smem <= 192 * 1024 &&
+      k + (shared_rows > 0 ? 1 : 0) <= 32) {
+    static SmemLimit lim;
+    const moe_status st = ensure_smem_limit(moe::scatter_rows_bulk_kernel, 192 * 1024, lim);
+    if (st != MOE_OK) return st;
+    const int per_sm = (int)std::max<size_t>(1, (160 * 1024) / bulk_smem);
+    const int grid = (int)std::min<int64_t>(n, (int64_t)sm_count() * std::min(per_sm, 8));
+    moe::scatter_rows_bulk_kernel<<<grid, 32, bulk_smem, s>>>((const uint8_t*)xn, slot_row, offsets, e, n, k,
+                                                             (uint8_t*)x_perm, (uint32_t)row_bytes, shared_rows,
+                                                             hdr, wait_limit_ns());
+    return launch_status();
+  }
   // columns counted in 16-byte vectors, or elements for the narrower forms
   const int vec_elems = (row_bytes % 16 == 0 && addr % 16 == 0) ? (dtype == MOE_BF16 ? 8 : 4) : 1;
   const dim3 grid = row_split_grid(n, d, vec_elems);
