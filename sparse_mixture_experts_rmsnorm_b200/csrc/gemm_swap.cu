@@ -46,7 +46,13 @@
 //               stores.
 // Tiles run group by group; within a group, chunks in runs of eight share
 // the walk over the weight tiles, so the SM pairs that hold one weight tile's
-// chunks run at the same time.  No TMA load uses cluster multicast.  Every
+// chunks run at the same time.  Each pair claims its next tile from a
+// per-launch counter and hands the index to the other roles through a ring.
+// Data that crosses to the other CTA (ring entries, SwiGLU halves) travels by
+// st.async, counted on the receiving barrier, and slots are handed back with
+// relaxed arrivals: a cluster-scope release would hold the arriving thread
+// until its earlier memory operations are performed at cluster scope, about
+// 1.4 k cycles each time on B200.  No TMA load uses cluster multicast.  Every
 // mbarrier wait is bounded: on time-out the block records
 // MOE_ERR_DEVICE_TIMEOUT, stops issuing work, drains and returns; both CTAs
 // always meet at the final cluster barrier.
