@@ -173,7 +173,10 @@ moe_status moe_route_hash(const moe_config* cfg, const void* h, const void* norm
  *   offsets   [E+1]  out: offsets[e] = sum of kept counts of experts < e
  *   slot_row  [N*k]  out
  *   row_token [N*k]  out (first offsets[E] entries valid)
- *   x_perm    [R][d] out: x_perm[slot_row[s]] = xn[s / k] for kept slots */
+ *   x_perm    [R][d] out: x_perm[slot_row[s]] = xn[s / k] for kept slots
+ * The gather's device-side waits (on its bulk row copies) are bounded by
+ * moe_set_wait_timeout_ns; a time-out is recorded in the workspace error
+ * word (moe_check_device_error). */
 moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* xn, int32_t* offsets,
                        int32_t* slot_row, int32_t* row_token, void* x_perm, void* ws, size_t ws_bytes,
                        void* stream);
@@ -201,7 +204,9 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const voi
  *    device's primary context: after cudaDeviceReset, or with another
  *    driver-API context current, the call is not supported;
  *  - every call on a device shares the one array: calls that overlap on the
- *    GPU (other streams, other threads) race and give wrong results.
+ *    GPU (other streams, other threads) race and give wrong results;
+ *  - with no workspace there is no error word: a device-side wait of the
+ *    gather that runs out (see moe_permute) ends its block without a record.
  * The call allocates nothing and frees nothing. */
 moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* topk_idx, const void* xn, int32_t* offsets,
                                int32_t* slot_row, int32_t* row_token, void* x_perm, void* stream);
