@@ -337,7 +337,14 @@ def run_native(args):
 
     e2e_steps(max(2, args.warmup // 2))
     torch.cuda.synchronize()
-    e_steps = max(3, args.steps // 2)
+    # the same untimed pre-roll as before the device-only region: staging the
+    # pinned input above leaves the GPU idle long enough for its clock to
+    # recover, which would flatter the first timed steps
+    pre = preroll_steps(lambda: e2e_steps(1), args.preroll)
+    pre = int(max_over_ranks([pre], "cuda")[0]) - pre
+    for _ in range(pre):
+        e2e_steps(1)
+    e_steps = max(3, args.steps)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
