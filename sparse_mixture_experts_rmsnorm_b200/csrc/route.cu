@@ -322,8 +322,10 @@ static moe_status launch_rr(const void* h, const void* norm_w, const void* w_rou
   }
   const int epb = (logits == nullptr) ? 1 : (e <= 32 ? e : 32);
   const int yb = (logits == nullptr) ? 1 : (e + epb - 1) / epb;
+  // RMSNorm alone: 128-thread blocks, so twice as many tokens are in flight per SM
+  const int threads = logits == nullptr ? 128 : 256;
   int xb = n < sm_count() * 16 ? n : sm_count() * 16;
-  kern<<<dim3(xb, yb), 256, smem, s>>>((const T*)h, (const T*)norm_w, (const T*)w_router, (T*)xn, logits, n, d, e,
+  kern<<<dim3(xb, yb), threads, smem, s>>>((const T*)h, (const T*)norm_w, (const T*)w_router, (T*)xn, logits, n, d, e,
                                        epb, eps);
   return launch_status();
 }
