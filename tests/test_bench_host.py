@@ -81,6 +81,6 @@ def test_set_overrides_keep_field_types():
 def test_traffic_figure_belongs_to_the_current_gemm_sources():
     # the ratio is reported only while the GEMM sources hash to the captured one
     assert bench.TRAFFIC["kernel_sha"] == bench._kernel_sha(), (
-        "the GEMM sources changed since the DRAM traffic capture: take it again on the 32-expert case "
-        "(profiles/gemm_swap_dsv3_prefill_shape.md) and update bench.TRAFFIC")
+        "the GEMM sources changed since the DRAM traffic capture: take it again on the 32-expert "
+        "DeepSeek-V3-shaped case and update bench.TRAFFIC")
     assert 0.9 < bench.TRAFFIC["per_algorithmic_byte"] < 1.2
