@@ -49,7 +49,8 @@ UNIT = "tokens/s"
 # applied to the full launch's algorithmic bytes: both are dominated by the
 # touched experts' weights, which every launch reads once.
 TRAFFIC = {"kernel_sha": "f929f29a69c46967", "workload": "dsv3_prefill_bf16", "per_algorithmic_byte": 1.0211,
-           "source": "profiles/gemm_swap_dsv3_prefill_shape.md (E = 32, N = 1024 case, scaled)"}
+           "source": "ncu DRAM bytes of the gate/up launch on the E = 32, N = 1024 case of the same per-expert "
+                     "shape, per algorithmic byte, times this launch's algorithmic bytes"}
 
 
 def _peaks():
