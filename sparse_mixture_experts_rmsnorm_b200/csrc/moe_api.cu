@@ -167,8 +167,7 @@ static moe_status permute_impl(const moe_config* c, const int32_t* topk_idx, con
   const int cap = (int)capacity_of(c);
   MOE_TRY(launch_permute(topk_idx, c->n_tokens, c->top_k, c->n_experts, cap, (int32_t*)wsp(ws, L.hist), offsets,
                          slot_row, row_token, s, nullptr, 0, counts));
-  return launch_gather(c->dtype, xn, slot_row, offsets, c->n_experts, c->n_tokens, c->top_k, x_perm, c->d_model, s,
-                       0, (int32_t*)wsp(ws, L.hdr));
+  return launch_gather(c->dtype, xn, slot_row, c->n_tokens, c->top_k, x_perm, c->d_model, s, (int32_t*)wsp(ws, L.hdr));
 }
 
 static moe_status ffn_impl(const moe_config* c, int groups, const int32_t* offsets, int max_rows, const void* x,
@@ -317,8 +316,7 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const 
     int32_t* offs_ext = (int32_t*)wsp(ws, L.offsets_ext);
     MOE_TRY(launch_permute(idx, N, cfg->top_k, cfg->n_experts, (int)capacity_of(cfg), (int32_t*)wsp(ws, L.hist),
                            offsets, slot_row, row_token, s, offs_ext, N, counts));
-    MOE_TRY(launch_gather(cfg->dtype, xn, slot_row, offsets, cfg->n_experts, N, cfg->top_k, x_perm, cfg->d_model, s,
-                          0, hdr));
+    MOE_TRY(launch_gather(cfg->dtype, xn, slot_row, N, cfg->top_k, x_perm, cfg->d_model, s, hdr));
     MOE_TRY(mark(trace ? trace->permuted : nullptr));
     if (N > 0) {
       MOE_TRY(launch_gemm_tc(EPI_SWIGLU, x_perm, w->w_gate, w->w_up, offs_ext, cfg->n_experts + 1, R + N, cfg->d_ff,

@@ -44,12 +44,11 @@ moe_status launch_permute(const int32_t* topk_idx, int n, int k, int e, int cap,
                           int32_t* offsets_ext = nullptr, int extra = 0, int32_t* counts = nullptr);
 
 // a5: x_perm[slot_row[t * k + j]] = xn[t] for every kept slot (that is,
-// x_perm[r] = xn[row_token[r]] for r < R = offsets[e], a device count), and
-// x_perm[R + t] = xn[t] for t < shared_rows (the folded shared expert).
+// x_perm[r] = xn[row_token[r]] for r < R = offsets[e], a device count).
 // Token order: each xn row is read once.  k <= 32.  hdr: the workspace's
 // error word for the bounded waits of the bulk-copy form (may be null).
-moe_status launch_gather(int dtype, const void* xn, const int32_t* slot_row, const int32_t* offsets, int e, int n,
-                         int k, void* x_perm, int d, cudaStream_t s, int shared_rows = 0, int32_t* hdr = nullptr);
+moe_status launch_gather(int dtype, const void* xn, const int32_t* slot_row, int n, int k, void* x_perm, int d,
+                         cudaStream_t s, int32_t* hdr = nullptr);
 
 // a9: out = h + sum_j gate_j * y_perm[slot_row] (+ y_shared).  With
 // shared_offsets != nullptr the shared rows are y_perm rows from

@@ -286,9 +286,9 @@ __global__ void __launch_bounds__(1024) permute_fused_kernel(const int32_t* __re
 }
 
 // a5 in token order: token t's row of xn is read once and written to each
-// of its kept slots, x_perm[slot_row[t * k + j]] = xn[t], and, with
-// shared_rows > 0, to x_perm[R + t] (R = offsets[E]) for the folded shared
-// expert.  Every x_perm row r < R has exactly one kept slot pointing at it,
+// of its kept slots, x_perm[slot_row[t * k + j]] = xn[t].  (A folded shared
+// expert reads its rows straight from xn.)  Every x_perm row r < R has
+// exactly one kept slot pointing at it,
 // so this writes the same x_perm as reading x_perm[r] = xn[row_token[r]],
 // while each xn row crosses HBM once instead of once per slot.  One block
 // per token (grid-stride); VEC elements per 16-byte access when the row
@@ -296,24 +296,20 @@ __global__ void __launch_bounds__(1024) permute_fused_kernel(const int32_t* __re
 template <typename V>
 __global__ void __launch_bounds__(128) scatter_rows_kernel(const V* __restrict__ xn,
                                                            const int32_t* __restrict__ slot_row,
-                                                           const int32_t* __restrict__ offsets, int E, int n, int k,
-                                                           V* __restrict__ x_perm, int row_vecs, int shared_rows) {
-  __shared__ int32_t dst[33];
-  const int routed = offsets[E];
-  const int nd = k + (shared_rows > 0 ? 1 : 0);
+                                                           int n, int k, V* __restrict__ x_perm, int row_vecs) {
+  __shared__ int32_t dst[32];
   // block (x, y): tokens x, x + gridDim.x, ..., the y-th column range of each row
   const int w = (row_vecs + (int)gridDim.y - 1) / (int)gridDim.y;
   const int ib = min(row_vecs, (int)blockIdx.y * w);
   const int ie = min(row_vecs, ib + w);
   for (int t = blockIdx.x; t < n; t += gridDim.x) {
     if (threadIdx.x < k) dst[threadIdx.x] = slot_row[(size_t)t * k + threadIdx.x];
-    if (threadIdx.x == 0 && shared_rows > 0) dst[k] = t < shared_rows ? routed + t : -1;
     __syncthreads();
     const V* src = xn + (size_t)t * row_vecs;
 #pragma unroll 4
     for (int i = ib + threadIdx.x; i < ie; i += blockDim.x) {
       const V v = src[i];
-      for (int j = 0; j < nd; ++j) {
+      for (int j = 0; j < k; ++j) {
         const int r = dst[j];
         if (r >= 0) x_perm[(size_t)r * row_vecs + i] = v;
       }
@@ -326,8 +322,8 @@ __global__ void __launch_bounds__(128) scatter_rows_kernel(const V* __restrict__
 // SM only issues them).  One warp per block; lane 0 keeps kBulkRing rows of
 // the block's tokens (t = blockIdx.x, + gridDim.x, ...) in flight: each row
 // arrives in shared memory by one bulk load completing on that buffer's
-// mbarrier, then leaves by one bulk store per kept slot (and the shared
-// expert's row), committed as one bulk group.  A buffer is reloaded once the
+// mbarrier, then leaves by one bulk store per kept slot, committed as one
+// bulk group.  A buffer is reloaded once the
 // group that read it has finished reading (wait_group.read).  Lane j < nd
 // holds destination j of the next token, loaded a token ahead.  Rows must be
 // 16-byte aligned and a multiple of 16 bytes.
@@ -335,15 +331,12 @@ constexpr int kBulkRing = 4;
 
 __global__ void __launch_bounds__(32) scatter_rows_bulk_kernel(const uint8_t* __restrict__ xn,
                                                                const int32_t* __restrict__ slot_row,
-                                                               const int32_t* __restrict__ offsets, int E, int n,
-                                                               int k, uint8_t* __restrict__ x_perm,
-                                                               uint32_t row_bytes, int shared_rows,
-                                                               int32_t* __restrict__ hdr, uint64_t wait_ns) {
+                                                               int n, int k, uint8_t* __restrict__ x_perm,
+                                                               uint32_t row_bytes, int32_t* __restrict__ hdr,
+                                                               uint64_t wait_ns) {
   extern __shared__ __align__(128) uint8_t rows[];
   __shared__ __align__(8) uint64_t full[kBulkRing];
   const int lane = lane_id();
-  const int routed = offsets[E];
-  const int nd = k + (shared_rows > 0 ? 1 : 0);
   const int64_t count = (n - (int64_t)blockIdx.x + gridDim.x - 1) / gridDim.x;  // this block's tokens
   if (lane == 0) {
     for (int b = 0; b < kBulkRing; ++b) mbar_init(&full[b], 1);
@@ -352,10 +345,8 @@ __global__ void __launch_bounds__(32) scatter_rows_bulk_kernel(const uint8_t* __
   __syncwarp();
   auto token = [&](int64_t i) { return (int64_t)blockIdx.x + i * gridDim.x; };
   auto dst_of = [&](int64_t i) -> int {  // this lane's destination of the block's i-th token, or -1
-    if (i >= count || lane >= nd) return -1;
-    const int64_t t = token(i);
-    if (lane < k) return slot_row[t * k + lane];
-    return t < shared_rows ? routed + (int)t : -1;
+    if (i >= count || lane >= k) return -1;
+    return slot_row[token(i) * k + lane];
   };
   auto load = [&](int64_t i) {
     if (lane != 0 || i >= count) return;
@@ -378,7 +369,7 @@ __global__ void __launch_bounds__(32) scatter_rows_bulk_kernel(const uint8_t* __
       landed = mbar_wait_bounded(&full[b], (uint32_t)((i / kBulkRing) & 1), wait_ns, nullptr, hdr, KID_SCATTER, 1);
     if (!__shfl_sync(0xffffffffu, landed, 0)) break;
     const uint32_t src = smem_u32(rows + (size_t)b * row_bytes);
-    for (int j = 0; j < nd; ++j) {
+    for (int j = 0; j < k; ++j) {
       const int r = __shfl_sync(0xffffffffu, d_cur, j);
       if (lane == 0 && r >= 0)
         asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(x_perm +
@@ -445,8 +436,8 @@ moe_status launch_permute(const int32_t* topk_idx, int n, int k, int e, int cap,
   return launch_status();
 }
 
-moe_status launch_gather(int dtype, const void* xn, const int32_t* slot_row, const int32_t* offsets, int e, int n,
-                         int k, void* x_perm, int d, cudaStream_t s, int shared_rows, int32_t* hdr) {
+moe_status launch_gather(int dtype, const void* xn, const int32_t* slot_row, int n, int k, void* x_perm, int d,
+                         cudaStream_t s, int32_t* hdr) {
   if (n == 0) return MOE_OK;
   if (k > 32) return MOE_ERR_UNSUPPORTED;
   const size_t row_bytes = (size_t)d * (dtype == MOE_BF16 ? 2 : 4);
@@ -454,30 +445,28 @@ moe_status launch_gather(int dtype, const void* xn, const int32_t* slot_row, con
   // Bulk copies once there are enough tokens to keep every SM's copies busy
   // (the block-per-token kernel below splits rows over blocks for fewer).
   const size_t bulk_smem = moe::kBulkRing * row_bytes;
-  if (row_bytes % 16 == 0 && addr % 16 == 0 && n >= 2 * sm_count() && bulk_smem <= 192 * 1024 &&
-      k + (shared_rows > 0 ? 1 : 0) <= 32) {
+  if (row_bytes % 16 == 0 && addr % 16 == 0 && n >= 2 * sm_count() && bulk_smem <= 192 * 1024) {
     static SmemLimit lim;
     const moe_status st = ensure_smem_limit(moe::scatter_rows_bulk_kernel, 192 * 1024, lim);
     if (st != MOE_OK) return st;
     const int per_sm = (int)std::max<size_t>(1, (160 * 1024) / bulk_smem);
     const int grid = (int)std::min<int64_t>(n, (int64_t)sm_count() * std::min(per_sm, 8));
-    moe::scatter_rows_bulk_kernel<<<grid, 32, bulk_smem, s>>>((const uint8_t*)xn, slot_row, offsets, e, n, k,
-                                                             (uint8_t*)x_perm, (uint32_t)row_bytes, shared_rows,
-                                                             hdr, wait_limit_ns());
+    moe::scatter_rows_bulk_kernel<<<grid, 32, bulk_smem, s>>>((const uint8_t*)xn, slot_row, n, k, (uint8_t*)x_perm,
+                                                             (uint32_t)row_bytes, hdr, wait_limit_ns());
     return launch_status();
   }
   // columns counted in 16-byte vectors, or elements for the narrower forms
   const int vec_elems = (row_bytes % 16 == 0 && addr % 16 == 0) ? (dtype == MOE_BF16 ? 8 : 4) : 1;
   const dim3 grid = row_split_grid(n, d, vec_elems);
   if (row_bytes % 16 == 0 && addr % 16 == 0)
-    moe::scatter_rows_kernel<uint4><<<grid, 128, 0, s>>>((const uint4*)xn, slot_row, offsets, e, n, k,
-                                                         (uint4*)x_perm, (int)(row_bytes / 16), shared_rows);
+    moe::scatter_rows_kernel<uint4><<<grid, 128, 0, s>>>((const uint4*)xn, slot_row, n, k,
+                                                         (uint4*)x_perm, (int)(row_bytes / 16));
   else if (row_bytes % 4 == 0 && addr % 4 == 0)
-    moe::scatter_rows_kernel<uint32_t><<<grid, 128, 0, s>>>((const uint32_t*)xn, slot_row, offsets, e, n, k,
-                                                            (uint32_t*)x_perm, (int)(row_bytes / 4), shared_rows);
+    moe::scatter_rows_kernel<uint32_t><<<grid, 128, 0, s>>>((const uint32_t*)xn, slot_row, n, k,
+                                                            (uint32_t*)x_perm, (int)(row_bytes / 4));
   else
-    moe::scatter_rows_kernel<uint16_t><<<grid, 128, 0, s>>>((const uint16_t*)xn, slot_row, offsets, e, n, k,
-                                                            (uint16_t*)x_perm, (int)(row_bytes / 2), shared_rows);
+    moe::scatter_rows_kernel<uint16_t><<<grid, 128, 0, s>>>((const uint16_t*)xn, slot_row, n, k,
+                                                            (uint16_t*)x_perm, (int)(row_bytes / 2));
   return launch_status();
 }
 

@@ -85,6 +85,5 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
   st = launch_permute(topk_idx, cfg->n_tokens, cfg->top_k, cfg->n_experts, (int)cap, hist, offsets, slot_row,
                       row_token, s);
   if (st != MOE_OK) return st;
-  return launch_gather(cfg->dtype, xn, slot_row, offsets, cfg->n_experts, cfg->n_tokens, cfg->top_k, x_perm,
-                       cfg->d_model, s);
+  return launch_gather(cfg->dtype, xn, slot_row, cfg->n_tokens, cfg->top_k, x_perm, cfg->d_model, s);
 }
