@@ -42,13 +42,14 @@ METRIC = "MoE-layer fwd tokens/s; expert GEMM TFLOP/s & HBM GB/s vs B200 peak"
 UNIT = "tokens/s"
 
 # DRAM bytes (read + write) of one launch of the dominant kernel, from an ncu
-# capture, with the sha256 of the kernel sources it was taken on; reported
+# capture, with the sha256 of that kernel's sources (the swapped-operand
+# kernel that runs every bf16 gate/up projection) it was taken on; reported
 # only while those sources are unchanged.  The full DeepSeek-V3-shaped
 # prefill holds too much on the device for a multi-pass capture, so its
 # figure is the 32-expert case's DRAM bytes per algorithmic byte (1.0211),
 # applied to the full launch's algorithmic bytes: both are dominated by the
 # touched experts' weights, which every launch reads once.
-TRAFFIC = {"kernel_sha": "f929f29a69c46967", "workload": "dsv3_prefill_bf16", "per_algorithmic_byte": 1.0211,
+TRAFFIC = {"kernel_sha": "7d6f90d28f99f4f8", "workload": "dsv3_prefill_bf16", "per_algorithmic_byte": 1.0211,
            "source": "ncu DRAM bytes of the gate/up launch on the E = 32, N = 1024 case of the same per-expert "
                      "shape, per algorithmic byte, times this launch's algorithmic bytes"}
 
@@ -70,14 +71,16 @@ def _dist():
 
 
 GEMM_SOURCES = ("gemm_tc.cu", "gemm_tc2.cu", "gemm_swap.cu", "tcgen05.cuh", "tcgen05_pair.cuh")
+GATE_UP_SOURCES = ("gemm_swap.cu", "tcgen05.cuh", "tcgen05_pair.cuh")
 
 
-def _kernel_sha():
-    """sha256 prefix of the code of the grouped GEMM kernels: their source
-    files with `//` comments, trailing blanks and empty lines removed, so that a
-    comment edit does not retire a traffic figure."""
+def _kernel_sha(sources=GATE_UP_SOURCES):
+    """sha256 prefix of the code of the given kernel sources (by default the
+    gate/up kernel's): the files with `//` comments, trailing blanks and
+    empty lines removed, so that a comment edit does not retire a traffic
+    figure."""
     h = hashlib.sha256()
-    for name in GEMM_SOURCES:
+    for name in sources:
         with open(os.path.join(ROOT, "sparse_mixture_experts_rmsnorm_b200", "csrc", name), encoding="utf-8") as f:
             for line in f:
                 code = line.split("//", 1)[0].rstrip()

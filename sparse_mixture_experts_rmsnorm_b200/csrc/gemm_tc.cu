@@ -30,6 +30,16 @@
 // units, so one N = 256 MMA produces both halves.  A plain-epilogue launch
 // with too few tiles to fill the SMs (the router's logits) uses 128-column
 // tiles: one B box per stage and N = 128 MMAs.
+// The fp32 epilogue (router logits) always runs 128-column tiles and
+// accumulates in K-chunks.  The tensor cores' fp32 accumulator loses more
+// per step than a round-to-nearest add: measured on B200 against a float64
+// router with K = 7168 and 256 experts, one accumulator per tile put the
+// selection keys (softmax score + bias) off by up to 1.2e-5, enough to swap
+// two experts whose keys differ by 1.1e-6; chunks of 256 (or 128) along K
+// bring that to 6.6e-7, and chunks of 512 to 8.9e-7.  So each chunk of
+// TC_F32_CHUNK_KB k-blocks starts a fresh accumulator in one of four
+// 128-column TMEM slots, and the epilogue warps add the chunks in order in
+// fp32 registers (round-to-nearest) before the single store of the row.
 // Tiles are numbered group-major, then n-tile, then m-tile, so CTAs working
 // at the same time share weight tiles through L2.
 // Every mbarrier wait is bounded: on time-out the block records
@@ -52,6 +62,24 @@ constexpr int TC_STAGE_BYTES = TC_A_BYTES + 2 * TC_B_HALF_BYTES;
 constexpr int TC_EPI_STAGE_BYTES = 32 * 128;  // one warp's 32 x 64 bf16 output block (TMA-store epilogue)
 constexpr int TC_SMEM_BYTES = TC_STAGES * TC_STAGE_BYTES + 4 * TC_EPI_STAGE_BYTES + 1024;  // + alignment slack
 constexpr int TC_THREADS = 192;
+constexpr int TC_F32_CHUNK_KB = 4;  // k-blocks (of 64) per fp32 partial accumulator: K = 256
+
+// Writes one fp32 row of 128 columns n0 .. n0 + 127, masked to columns < nout.
+__device__ __forceinline__ void store_row128_f32(const TcArgs& args, int row, int n0, const float (&v)[128]) {
+  float* out = reinterpret_cast<float*>(args.C) + (size_t)row * args.ldc;
+  const bool vec = (args.ldc & 3) == 0 && (reinterpret_cast<uintptr_t>(args.C) & 15) == 0;
+#pragma unroll
+  for (int c = 0; c < 128; c += 4) {
+    const int col = n0 + c;
+    if (vec && col + 4 <= args.nout) {
+      *reinterpret_cast<float4*>(out + col) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        if (col + i < args.nout) out[col + i] = v[c + i];
+    }
+  }
+}
 
 template <int EPI>
 __global__ void __launch_bounds__(TC_THREADS, 1)
@@ -62,8 +90,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[TC_STAGES];
   __shared__ __align__(8) uint64_t empty_bar[TC_STAGES];
-  __shared__ __align__(8) uint64_t tfull_bar[2];
-  __shared__ __align__(8) uint64_t tempty_bar[2];
+  // accumulator slots: two of 256 columns (one per tile), or four of 128
+  // columns (one per K-chunk) for the fp32 epilogue
+  constexpr bool F32 = EPI == moe_host::EPI_F32;
+  constexpr int NBUF = F32 ? 4 : 2;
+  constexpr uint32_t SLOT_COLS = F32 ? 128u : (uint32_t)TC_BN;
+  __shared__ __align__(8) uint64_t tfull_bar[NBUF];
+  __shared__ __align__(8) uint64_t tempty_bar[NBUF];
   __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
@@ -95,7 +128,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NBUF; ++b) {
       mbar_init(&tfull_bar[b], 1);
       mbar_init(&tempty_bar[b], 4);
     }
@@ -114,6 +147,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const uint32_t tmem_base = tmem_base_sh;
   const int total_tiles = prefix_sh[G];
   const int nk = (args.K + TC_BK - 1) / TC_BK;
+  // k-blocks per accumulator and accumulators per tile
+  const int chunk_kb = F32 ? TC_F32_CHUNK_KB : nk;
+  const int n_chunks = F32 ? (nk + TC_F32_CHUNK_KB - 1) / TC_F32_CHUNK_KB : 1;
 
   if (warp == 0) {
     // ======================= TMA producer =======================
@@ -177,7 +213,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   } else if (warp == 1) {
     // ======================= MMA issuer =======================
     if (lane == 0) {
-      // 128-column tiles (plain epilogues with few tiles) run N = 128 MMAs
+      // 128-column tiles (the fp32 epilogue, and plain stores with few tiles) run N = 128 MMAs
       const int bn = (EPI != moe_host::EPI_SWIGLU && args.narrow) ? 128 : TC_BN;
       const uint32_t idesc = tc_idesc(TC_BM, bn);
       int stage = 0;
@@ -189,35 +225,41 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const Tile tl = decode_tile<TC_BM>(t, prefix_sh, offs_sh, G, args.out_cols);
         // a tile of at most 64 rows runs as M = 64 MMAs (half the rows of work)
         const uint32_t id = (tl.row_end - tl.row0 <= 64) ? tc_idesc(64, bn) : idesc;
-        if (!mbar_wait_bounded(&tempty_bar[buf], bphase ^ 1u, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
-                               SITE_TMEM_EMPTY))
-          break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(buf * TC_BN);
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait_bounded(&full_bar[stage], phase, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
-                                 SITE_FULL)) {
+        for (int c = 0; c < n_chunks && ok; ++c) {
+          if (!mbar_wait_bounded(&tempty_bar[buf], bphase ^ 1u, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
+                                 SITE_TMEM_EMPTY)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_base + stage * TC_STAGE_BYTES;
-          const uint64_t adesc = sw128_desc(sa);
-          const uint64_t bdesc = sw128_desc(sa + TC_A_BYTES);
+          const uint32_t d_tmem = tmem_base + (uint32_t)buf * SLOT_COLS;
+          const int kb0 = c * chunk_kb;
+          const int kb1 = kb0 + chunk_kb < nk ? kb0 + chunk_kb : nk;
+          for (int kb = kb0; kb < kb1; ++kb) {
+            if (!mbar_wait_bounded(&full_bar[stage], phase, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
+                                   SITE_FULL)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sa = smem_base + stage * TC_STAGE_BYTES;
+            const uint64_t adesc = sw128_desc(sa);
+            const uint64_t bdesc = sw128_desc(sa + TC_A_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < TC_BK / 16; ++kk)  // K = 16 per MMA: 32 bytes further along the row
-            tc_mma(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), id, (kb | kk) != 0);
-          tc_commit(&empty_bar[stage]);
-          if (++stage == TC_STAGES) {
-            stage = 0;
-            phase ^= 1u;
+            for (int kk = 0; kk < TC_BK / 16; ++kk)  // K = 16 per MMA: 32 bytes further along the row
+              tc_mma(d_tmem, adesc + (uint64_t)(kk * 2), bdesc + (uint64_t)(kk * 2), id, ((kb - kb0) | kk) != 0);
+            tc_commit(&empty_bar[stage]);
+            if (++stage == TC_STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
-        }
-        if (!ok) break;
-        tc_commit(&tfull_bar[buf]);
-        if (++buf == 2) {
-          buf = 0;
-          bphase ^= 1u;
+          if (!ok) break;
+          tc_commit(&tfull_bar[buf]);
+          if (++buf == NBUF) {
+            buf = 0;
+            bphase ^= 1u;
+          }
         }
       }
       // Drain: every MMA issued by this thread completes before TMEM is freed.
@@ -232,6 +274,42 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     uint32_t bphase = 0;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
       const Tile tl = decode_tile<TC_BM>(t, prefix_sh, offs_sh, G, args.out_cols);
+      if constexpr (F32) {
+        // the tile's K-chunks, summed in order in fp32 registers
+        const bool half = tl.row_end - tl.row0 <= 64;
+        const int row = half ? tl.row0 + quarter * 16 + (lane & 15) : tl.row0 + r_local;
+        float acc[128];
+#pragma unroll
+        for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
+        bool ok = true;
+        for (int c = 0; c < n_chunks; ++c) {
+          if (lane == 0)
+            ok = mbar_wait_bounded(&tfull_bar[buf], bphase, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
+                                   SITE_TMEM_FULL);
+          ok = __shfl_sync(0xffffffffu, ok, 0);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)buf * SLOT_COLS;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint32_t a[32];
+            MOE_TMEM_LD32(tb + 32 * j, a);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[32 * j + i] = __fadd_rn(acc[32 * j + i], __uint_as_float(a[i]));
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty_bar[buf]);
+          if (++buf == NBUF) {
+            buf = 0;
+            bphase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if (row < tl.row_end && (!half || lane < 16)) store_row128_f32(args, row, tl.n0, acc);
+        continue;
+      }
       bool ok = true;
       if (lane == 0)
         ok = mbar_wait_bounded(&tfull_bar[buf], bphase, args.wait_ns, &abort_flag, args.hdr, KID_GEMM_TC,
@@ -239,7 +317,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * TC_BN);
+      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)buf * SLOT_COLS;
       // M = 64 accumulators keep row r in lane (r / 16) * 32 + r % 16: lanes
       // 0..15 of each warp's quarter
       const bool half = tl.row_end - tl.row0 <= 64;
@@ -255,7 +333,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty_bar[buf]);
-      if (++buf == 2) {
+      if (++buf == NBUF) {
         buf = 0;
         bphase ^= 1u;
       }
@@ -432,20 +510,29 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
                          (epi == EPI_SWIGLU || (epi == EPI_STORE && rows_per_group >= 64));
   if ((forced == 3 || swap_auto) && swap_supported(epi, nout, k, ldc))
     return launch_gemm_swap(epi, a, b, b2, offsets, groups, max_rows, nout, k, c, ldc, hdr, s, sb, sb2, sa, sa_rows);
-  const int mode = forced == 3 ? 0 : forced;  // the router's fp32 logits: the automatic choice
   // Upper bound on the number of tiles; the exact count lives on the device.
   const int64_t m_tiles = (int64_t)(max_rows + moe::TC_BM - 1) / moe::TC_BM + (offsets ? groups : 0);
-  // A plain-epilogue launch that would leave more than half the SMs idle
-  // (the router's N x E logits: one 256-column tile per 128 rows) runs
+  if (epi == EPI_F32) {
+    // fp32 outputs (the router's logits) always take single-SM 128-column
+    // tiles, accumulated in K-chunks, whatever the tiling setting
+    args.narrow = 1;
+    args.out_cols = 128;
+    args.n_tiles = (nout + 127) / 128;
+    const int64_t tiles = m_tiles * args.n_tiles;
+    return launch_tc_t<EPI_F32>(ma, mb, mb2, msb, msb2, msa, mc, args, (int)(tiles < sm_count() ? tiles : sm_count()),
+                                s);
+  }
+  const int mode = forced == 3 ? 0 : forced;
+  // A plain-store launch that would leave more than half the SMs idle runs
   // 128-column tiles on single SMs instead, twice as many.
-  const bool few = epi != EPI_SWIGLU && mode != 2 && nout > 128 && m_tiles * args.n_tiles < sm_count() / 2;
+  const bool few = epi == EPI_STORE && mode != 2 && nout > 128 && m_tiles * args.n_tiles < sm_count() / 2;
   // Measured on B200: SM pairs help the plain-store epilogue of large groups
   // (down projection) by a few percent when both tilings take the same number
   // of waves; for the SwiGLU projection the extra padding of 256-row tiles
   // outweighs the saved operand traffic.  The group sizes live on the device,
   // so for the grouped down projection both kernels are launched and each
-  // keeps or drops itself from the offsets (pairs_picked); the router's
-  // single group keeps the host rule.
+  // keeps or drops itself from the offsets (pairs_picked); a single group
+  // keeps the host rule.
   const bool pair_rule = mode == 2 || (mode == 0 && rows_per_group >= 512 && epi != EPI_SWIGLU && !few);
   const bool device_pick = mode == 0 && pair_rule && epi == EPI_STORE && offsets != nullptr;
   if (pair_rule && !device_pick)
@@ -466,8 +553,7 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
     args.pick = 1;
   }
   if (epi == EPI_SWIGLU) return launch_tc_t<EPI_SWIGLU>(ma, mb, mb2, msb, msb2, msa, mc, args, grid, s);
-  if (epi == EPI_STORE) return launch_tc_t<EPI_STORE>(ma, mb, mb2, msb, msb2, msa, mc, args, grid, s);
-  return launch_tc_t<EPI_F32>(ma, mb, mb2, msb, msb2, msa, mc, args, grid, s);
+  return launch_tc_t<EPI_STORE>(ma, mb, mb2, msb, msb2, msa, mc, args, grid, s);
 }
 
 static std::atomic<int> g_pairing{0};

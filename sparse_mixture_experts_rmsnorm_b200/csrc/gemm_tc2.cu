@@ -277,8 +277,7 @@ static int resident_pairs() {
 
 static int resident_pairs_of(int epi) {
   if (epi == EPI_SWIGLU) return resident_pairs<EPI_SWIGLU>();
-  if (epi == EPI_STORE) return resident_pairs<EPI_STORE>();
-  return resident_pairs<EPI_F32>();
+  return resident_pairs<EPI_STORE>();
 }
 
 // Upper bound on the pair tiles (the exact count lives on the device).
@@ -313,7 +312,7 @@ moe_status launch_gemm_tc2(int epi, const CUtensorMap& ma, const CUtensorMap& mb
   const int64_t bound = pair_tile_bound(max_rows, groups_bound, args.n_tiles);
   if (epi == EPI_SWIGLU) return launch_tc2_t<EPI_SWIGLU>(ma, mb, mb2, msb, msb2, msa, mc, args, bound, s);
   if (epi == EPI_STORE) return launch_tc2_t<EPI_STORE>(ma, mb, mb2, msb, msb2, msa, mc, args, bound, s);
-  return launch_tc2_t<EPI_F32>(ma, mb, mb2, msb, msb2, msa, mc, args, bound, s);
+  return MOE_ERR_UNSUPPORTED;  // fp32 outputs run on the single-SM kernel only
 }
 
 }  // namespace moe_host

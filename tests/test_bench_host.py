@@ -4,8 +4,8 @@ The algorithmic FLOPs and bytes are counted here a second way, expert by
 expert from the routing's group sizes, and checked against the closed forms
 bench.py uses; the figures quoted for the DeepSeek-V3-shaped prefill (its
 kept-row count is fixed by the top-8 routing without a capacity) are checked
-as numbers.  The DRAM traffic figure is only reported on the GEMM sources it
-was captured on.
+as numbers.  The DRAM traffic figure is only reported on the gate/up kernel
+sources it was captured on.
 """
 import argparse
 import os
@@ -79,8 +79,8 @@ def test_set_overrides_keep_field_types():
 
 
 def test_traffic_figure_belongs_to_the_current_gemm_sources():
-    # the ratio is reported only while the GEMM sources hash to the captured one
+    # the ratio is reported only while the gate/up kernel's sources hash to the captured one
     assert bench.TRAFFIC["kernel_sha"] == bench._kernel_sha(), (
-        "the GEMM sources changed since the DRAM traffic capture: take it again on the 32-expert "
-        "DeepSeek-V3-shaped case and update bench.TRAFFIC")
+        "the gate/up kernel's sources changed since the DRAM traffic capture: take it again on the "
+        "32-expert DeepSeek-V3-shaped case and update bench.TRAFFIC")
     assert 0.9 < bench.TRAFFIC["per_algorithmic_byte"] < 1.2

@@ -1,4 +1,6 @@
-"""GPU parity of the four bf16 layer workloads at their full sizes.
+"""GPU parity of the four bf16 layer workloads at their full sizes, and of
+the DeepSeek-V3-shaped prefill at four times its tokens (N = 32768: full
+256-row chunks, 1024 permutation chunks, the largest layer the tests run).
 
 Routing, counts, permutation and drop masks are checked on every token;
 outputs on a stratified sample the oracle computes token by token (each
@@ -19,7 +21,8 @@ from parity_helpers import (BF16_REL_RMS, bf16_half_ulp, bf16_rel_rms_err, capac
 pytestmark = pytest.mark.gpu
 
 # random tokens sampled on top of the stratified ones
-SAMPLES = {"mixtral_bf16": 24, "dsv3_prefill_bf16": 32, "dsv3_decode_bf16": 64, "stress_bf16": 16}
+SAMPLES = {"mixtral_bf16": 24, "dsv3_prefill_bf16": 32, "dsv3_decode_bf16": 64, "stress_bf16": 16,
+           "dsv3_prefill_bf16@32768": 16}
 
 
 def stratified_tokens(offsets, row_token, eligible, n_tokens, rng, n_random, late=8):
@@ -48,7 +51,10 @@ def test_config_parity(name):
     import torch
     import sparse_mixture_experts_rmsnorm_b200 as moe
 
-    cfg = mi.CONFIGS[name]
+    base, _, n_tokens = name.partition("@")
+    cfg = mi.CONFIGS[base]
+    if n_tokens:
+        cfg = cfg.with_(n_tokens=int(n_tokens))
     N, E, k = cfg.n_tokens, cfg.n_experts, cfg.top_k
     g = run_gpu_layer(cfg)
     ref = oracle_routing(cfg)
@@ -106,7 +112,7 @@ def test_config_parity(name):
         kept = np.diff(g["offsets"])
         assert np.all(kept <= cap)
 
-    if name == "stress_bf16":
+    if base == "stress_bf16":
         top1_share = float(np.mean(g["topk_idx"][:, 0] == 3))
         assert abs(top1_share - 0.90) <= 0.011, top1_share
         target = np.float32(N * k / E)
