@@ -83,7 +83,7 @@ def test_balancing_loop_on_the_stress_skew():
     # choices on expert 3), fifty route + bias-update iterations with
     # gamma = 1e-3 in one CUDA graph.  Biases must equal the oracle's bit for
     # bit after every iteration; counts too, except for tokens whose oracle
-    # keys at that iteration's bias are within 1e-6 (the router's fp32 sums
+    # keys at that iteration's bias are within KEY_TIE (the router's fp32 sums
     # may order those either way, and a count only moves the bias when it
     # crosses the target).
     import torch

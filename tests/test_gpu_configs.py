@@ -14,7 +14,7 @@ import pytest
 
 import moe_inputs as mi
 import oracle
-from parity_helpers import (BF16_REL_RMS, bf16_half_ulp, bf16_rel_rms_err, capacity, check_permutation,
+from parity_helpers import (BF16_REL_RMS, KEY_TIE, bf16_half_ulp, bf16_rel_rms_err, capacity, check_permutation,
                             check_routing, oracle_outputs, oracle_routing, rel_rms_err, run_gpu_layer, tie_masks,
                             to_np)
 
@@ -59,6 +59,11 @@ def test_config_parity(name):
     g = run_gpu_layer(cfg)
     ref = oracle_routing(cfg)
     np.testing.assert_array_equal(g["xn"], ref["xn"])
+    # the premise of the tie window: every fp32 selection key within KEY_TIE / 2 of the oracle's
+    bias32 = mi.host_tensor(cfg, "bias").astype(np.float32)
+    key_err = float(np.max(np.abs((g["scores"].astype(np.float32) + bias32[None, :]).astype(np.float64)
+                                  - ref["key"])))
+    assert key_err <= KEY_TIE / 2, key_err
     skipped = check_routing(g, ref, k)
     assert skipped <= max(2, 0.01 * N), skipped
     cap = capacity(cfg)
@@ -101,7 +106,7 @@ def test_config_parity(name):
           f"{bs_delta:.3e}; rms(out) = {np.sqrt(np.mean(ref_out ** 2)):.3f}, rms(out-h) = {delta_rms:.4f}; "
           f"tokens {tokens.size}, experts covered "
           f"{covered.size} of {E}{' + shared' if cfg.d_ff_shared else ''}, skipped ties {skipped}, "
-          f"dropped slots {int((~gpu_keep).sum())}")
+          f"dropped slots {int((~gpu_keep).sum())}, max key err {key_err:.2e}")
     assert err <= BF16_REL_RMS, err
 
     if cap >= 0:
