@@ -339,17 +339,16 @@ moe_status launch_gemm_swap(int epi, const void* a, const void* b, const void* b
 // SM pairs that launch_gemm_tc2 launches for these sizes.
 int64_t tc2_pairs_launched(int epi, int64_t max_rows, int groups_bound, int n_tiles);
 
-// 3: the swapped-operand SM-pair kernel for the expert GEMMs it supports
-//    (the rest, and the router, take 0's choice);
-// 0: choose per launch (the swapped-operand kernel, where it supports the
-//    shape, for the grouped plain store of groups averaging >= 64 rows and
-//    for SwiGLU over 16 or more groups averaging 64 .. 511 rows; single-SM
-//    tiles for the other SwiGLU launches; for the grouped plain store of groups
-//    averaging >= 512 rows both kernels are launched and the device picks
-//    from the group sizes (pairs_picked); the router's single group takes SM
-//    pairs from 512 rows);
-// 1: single-SM tiles only; 2: SM-pair tiles only; 3: swapped-operand SM-pair
-//    tiles for the expert GEMMs (the router's fp32 logits keep 0's choice).
+// 0: choose per launch: the swapped-operand SM-pair kernel, where it supports
+//    the shape, for every grouped SwiGLU launch and for the grouped plain store
+//    of groups averaging >= 64 rows; otherwise single-SM tiles, except that a
+//    plain store averaging >= 512 rows a group takes SM-pair tiles (when
+//    grouped, both kernels are launched and the device picks from the group
+//    sizes, pairs_picked);
+// 1: single-SM tiles only; 2: SM-pair tiles only; 3: the swapped-operand
+//    kernel for the expert GEMMs it supports (the rest take 0's choice).
+// The fp32 logits (the router) always take single-SM 128-column tiles with
+// K-chunked accumulation, whatever the mode.
 void set_tc_pairing(int mode);
 int tc_pairing();
 }  // namespace moe_host
