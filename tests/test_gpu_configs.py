@@ -1,6 +1,8 @@
 """GPU parity of the four bf16 layer workloads at their full sizes, and of
-the DeepSeek-V3-shaped prefill at four times its tokens (N = 32768: full
-256-row chunks, 1024 permutation chunks, the largest layer the tests run).
+the DeepSeek-V3-shaped prefill at four and eight times its tokens (N = 32768:
+full 256-row chunks, 1024 permutation chunks; N = 65536: the expert-sorted
+rows hold 3.76e9 elements, past 32-bit element offsets, the largest layer the
+tests run, about 45 GB on the device).
 
 Routing, counts, permutation and drop masks are checked on every token;
 outputs on a stratified sample the oracle computes token by token (each
@@ -22,7 +24,7 @@ pytestmark = pytest.mark.gpu
 
 # random tokens sampled on top of the stratified ones
 SAMPLES = {"mixtral_bf16": 24, "dsv3_prefill_bf16": 32, "dsv3_decode_bf16": 64, "stress_bf16": 16,
-           "dsv3_prefill_bf16@32768": 16}
+           "dsv3_prefill_bf16@32768": 16, "dsv3_prefill_bf16@65536": 16}
 
 
 def stratified_tokens(offsets, row_token, eligible, n_tokens, rng, n_random, late=8):
