@@ -221,6 +221,17 @@ def whole_job_tokens_per_s(tokens_per_rank: int, world: int, ms_per_step: float)
     return tokens_per_rank * world / (ms_per_step * 1e-3)
 
 
+def load_stats(moe, lc, counts, offsets):
+    """The library's load statistics of one routing (moe_compute_load_stats)."""
+    import ctypes
+    import torch
+    buf = torch.zeros(ctypes.sizeof(moe.MoeLoadStats), dtype=torch.uint8, device="cuda")
+    moe.moe_compute_load_stats(lc, counts, offsets, buf)
+    s = moe.MoeLoadStats.from_buffer_copy(bytes(buf.cpu().numpy()))
+    return {"routed_slots": s.routed, "kept_slots": s.kept, "dropped_slots": s.dropped, "max_count": s.max_count,
+            "max_over_mean": round(float(s.max_over_mean), 4)}
+
+
 def run_native(args):
     import numpy as np
     import torch
@@ -247,7 +258,8 @@ def run_native(args):
     ws = moe.workspace(lc)
     E = cfg.n_experts
     offsets = torch.zeros(E + 1, dtype=torch.int32, device="cuda")
-    routing = {"offsets": offsets}
+    counts = torch.zeros(E, dtype=torch.int32, device="cuda")
+    routing = {"offsets": offsets, "counts": counts}
     stream = torch.cuda.current_stream()
 
     def step(trace=None):
@@ -261,6 +273,7 @@ def run_native(args):
         raise RuntimeError(f"device error {info}")
     off_host = offsets.cpu().numpy()
     fb = workload_flops_bytes(cfg, off_host)
+    load = load_stats(moe, lc, counts, offsets)  # of this rank's routing, before the timed region
 
     # ---- timed region: K whole steps, per-stage events on the same stream
     names = ("start", "routed", "permuted", "gate_up", "down", "shared", "combined")
@@ -442,6 +455,7 @@ def run_native(args):
                             "frac_sustained": round(expert_tflops / peak_sus, 4), "ms": round(expert_ms, 4),
                             "flops": fb["expert_flops"], "kept_rows": fb["rows"]},
             "stage_ms": {n: round(v, 4) for n, v in stage.items()},
+            "load": load,
             "e2e": {"value": round(whole_job_tokens_per_s(cfg.n_tokens, world, e2e_ms), 1), "unit": UNIT,
                     "pipelining": "double-buffered: input copy, layer and output copy on three streams",
                     "h2d_bytes_per_step": h.numel() * h.element_size(),

@@ -255,6 +255,35 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* weights, 
 moe_status moe_bias_update(int32_t n_experts, const int32_t* counts, float target, float gamma, float* bias,
                            void* stream);
 
+/* Load statistics of one routing (steps a4 and a10).  Lesson "The
+ * load-balancing problem" (usage per expert against the target; with a
+ * capacity of C x N / E, overflow tokens pass the layer unprocessed) and
+ * "Step 2" (the usage that moves each bias); Ultralytics glossary "Load
+ * balancing and expert capacity" (tokens per expert counted; overflow
+ * continues on the residual).
+ *   routed        = N*k, the slots the top-k chose;
+ *   kept          = offsets[E], the slots that reached an expert;
+ *   dropped       = routed - kept (0 without a capacity);
+ *   max_count     = max over e of counts[e], taken before the capacity cut;
+ *   max_over_mean = fl32(max_count) / fl32(fl32(N*k) / fl32(E)), fp32
+ *                   divisions rounded to nearest (the mean load is the
+ *                   target usage N*k/E; 1 is perfect balance).
+ * counts [E] and offsets [E+1] are device int32 from moe_route / moe_permute
+ * or the moe_routing outputs of moe_layer_forward, for the same config;
+ * stats is one device moe_load_stats, written by one small kernel on
+ * `stream`.  MOE_ERR_INVALID_ARG for an invalid config or a NULL pointer
+ * (N = 0 writes routed = kept = dropped = max_count = 0, max_over_mean = 0). */
+typedef struct {
+  int32_t routed;
+  int32_t kept;
+  int32_t dropped;
+  int32_t max_count;
+  float max_over_mean;
+} moe_load_stats;
+
+moe_status moe_compute_load_stats(const moe_config* cfg, const int32_t* counts, const int32_t* offsets,
+                                  moe_load_stats* stats, void* stream);
+
 /* Synchronise `stream`, read and clear the workspace's device error word.
  * Returns MOE_OK, the recorded status (e.g. MOE_ERR_DEVICE_TIMEOUT) or
  * MOE_ERR_CUDA.  info (host, may be NULL) receives 4 int32 of detail

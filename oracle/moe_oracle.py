@@ -54,7 +54,7 @@ import numpy as np
 __all__ = [
     "round_to", "rmsnorm", "router_scores", "select_topk", "gates_from_scores",
     "expert_counts", "capacity_limit", "permute", "silu", "swiglu_expert",
-    "combine", "layer_forward", "bias_update", "balancing_loop", "splitmix64", "hash_route",
+    "combine", "layer_forward", "bias_update", "balancing_loop", "load_stats", "splitmix64", "hash_route",
 ]
 
 
@@ -264,6 +264,28 @@ def balancing_loop(scores, bias0, k: int, target: float, gamma: float, iteration
         counts.append(c)
         biases.append(bias.copy())
     return np.array(counts), np.array(biases)
+
+
+def load_stats(counts, offsets, n_tokens: int, top_k: int, n_experts: int) -> dict:
+    """Load statistics of one routing.
+
+    [LESSON] "The load-balancing problem" (each expert's usage against the
+    target N*k/E; with a capacity, overflow slots are dropped and pass the
+    layer) and [GLOSSARY] "Load balancing and expert capacity" (tokens per
+    expert counted; overflow continues on the residual).  routed = N*k
+    slots; kept = the slots the capacity let through (offsets[E]); dropped =
+    routed - kept; max_count = the largest count before the cut; and
+    max_over_mean = max_count over the mean load N*k/E, both divisions in
+    fp32 rounded to nearest, as the library defines it.  All zero for N = 0.
+    """
+    routed = int(n_tokens) * int(top_k)
+    if routed == 0:
+        return {"routed": 0, "kept": 0, "dropped": 0, "max_count": 0, "max_over_mean": np.float32(0.0)}
+    kept = int(np.asarray(offsets)[n_experts])
+    max_count = int(np.max(np.asarray(counts)))
+    mean = np.float32(np.float32(routed) / np.float32(n_experts))
+    return {"routed": routed, "kept": kept, "dropped": routed - kept, "max_count": max_count,
+            "max_over_mean": np.float32(np.float32(max_count) / mean)}
 
 
 # ----------------------------------------------------------------------------

@@ -31,7 +31,8 @@ MOE_F32, MOE_BF16 = 0, 1
 ENTRY_POINTS = (
     "moe_status_string", "moe_version", "moe_workspace_size", "moe_workspace_init", "moe_route", "moe_route_hash",
     "moe_permute", "moe_permute_noalloc", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_bias_update",
-    "moe_check_device_error", "moe_set_wait_timeout_ns", "moe_set_gemm_tiling", "moe_selftest_wait_timeout",
+    "moe_compute_load_stats", "moe_check_device_error", "moe_set_wait_timeout_ns", "moe_set_gemm_tiling",
+    "moe_selftest_wait_timeout",
 )
 
 
@@ -83,6 +84,7 @@ def _load():
         "moe_layer_forward": (I32, [cfgp, ctypes.POINTER(MoeWeights), P, P, P, ctypes.POINTER(MoeRouting),
                                     ctypes.POINTER(MoeTrace), P, SZ, P]),
         "moe_bias_update": (I32, [I32, P, F, F, P, P]),
+        "moe_compute_load_stats": (I32, [cfgp, P, P, P, P]),
         "moe_check_device_error": (I32, [P, SZ, P, P]),
         "moe_set_wait_timeout_ns": (I32, [I64]),
         "moe_set_gemm_tiling": (I32, [I32]),
@@ -248,6 +250,18 @@ def moe_layer_forward(cfg: Config, weights: dict, h, bias, out, ws, routing: dic
 def moe_bias_update(n_experts: int, counts, target: float, gamma: float, bias, stream=None):
     _check(_lib.moe_bias_update(n_experts, _ptr(counts), target, gamma, _ptr(bias), _stream(stream)),
            "moe_bias_update")
+
+
+class MoeLoadStats(ctypes.Structure):
+    """Host view of one moe_load_stats (20 bytes)."""
+    _fields_ = [("routed", ctypes.c_int32), ("kept", ctypes.c_int32), ("dropped", ctypes.c_int32),
+                ("max_count", ctypes.c_int32), ("max_over_mean", ctypes.c_float)]
+
+
+def moe_compute_load_stats(cfg: Config, counts, offsets, stats, stream=None):
+    """stats: a device buffer of at least ctypes.sizeof(MoeLoadStats) bytes."""
+    _check(_lib.moe_compute_load_stats(ctypes.byref(cfg.c()), _ptr(counts), _ptr(offsets), _ptr(stats),
+                                       _stream(stream)), "moe_compute_load_stats")
 
 
 def moe_check_device_error(ws, stream=None):

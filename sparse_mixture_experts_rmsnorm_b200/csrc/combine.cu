@@ -209,6 +209,32 @@ __global__ void bias_update_kernel(int E, const int32_t* __restrict__ counts, fl
   bias[e] = __fadd_rn(bias[e], __fmul_rn(s, gamma));
 }
 
+// Load statistics of one routing: routed = N*k slots, kept = offsets[E],
+// dropped = routed - kept, the largest pre-capacity count, and its ratio to
+// the mean load fl32(N*k) / fl32(E), each division rounded to nearest.
+__global__ void __launch_bounds__(256) load_stats_kernel(int slots, int E, const int32_t* __restrict__ counts,
+                                                         const int32_t* __restrict__ offsets,
+                                                         moe_load_stats* __restrict__ stats) {
+  __shared__ int warp_max[8];
+  int m = 0;
+  if (slots > 0)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) m = max(m, counts[e]);
+  m = __reduce_max_sync(0xffffffffu, m);
+  if (lane_id() == 0) warp_max[warp_id()] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int mx = 0;
+    for (int w = 0; w < (int)(blockDim.x / 32); ++w) mx = max(mx, warp_max[w]);
+    const int kept = slots > 0 ? offsets[E] : 0;
+    const float mean = __fdiv_rn((float)slots, (float)E);
+    stats->routed = slots;
+    stats->kept = kept;
+    stats->dropped = slots - kept;
+    stats->max_count = mx;
+    stats->max_over_mean = slots > 0 ? __fdiv_rn((float)mx, mean) : 0.f;
+  }
+}
+
 }  // namespace moe
 
 namespace moe_host {
@@ -250,6 +276,12 @@ moe_status launch_combine(int dtype, const void* h, const void* y_perm, const in
     else
       launch_combine_t<float, 1>(h, y_perm, slot_row, topk_gate, y_shared, out, n, d, k, shared_offsets, e, grid, s);
   }
+  return launch_status();
+}
+
+moe_status launch_load_stats(int slots, int e, const int32_t* counts, const int32_t* offsets, moe_load_stats* stats,
+                             cudaStream_t s) {
+  moe::load_stats_kernel<<<1, 256, 0, s>>>(slots, e, counts, offsets, stats);
   return launch_status();
 }
 

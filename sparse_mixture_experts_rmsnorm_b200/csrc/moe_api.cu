@@ -223,6 +223,7 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
 moe_status moe_route(const moe_config* cfg, const void* h, const void* norm_w, const void* w_router,
                      const float* bias, void* xn, float* scores, int32_t* topk_idx, float* topk_gate,
                      int32_t* counts, void* ws, size_t ws_bytes, void* stream) {
+  NvtxScope range("moe_route");
   MOE_TRY(check_common(cfg, ws, ws_bytes));
   if (cfg->n_tokens > 0 && (!h || !norm_w || !w_router || !xn || !topk_idx || !topk_gate)) return MOE_ERR_INVALID_ARG;
   if (!counts) return MOE_ERR_INVALID_ARG;
@@ -233,6 +234,7 @@ moe_status moe_route(const moe_config* cfg, const void* h, const void* norm_w, c
 moe_status moe_route_hash(const moe_config* cfg, const void* h, const void* norm_w, const int64_t* token_ids,
                           void* xn, int32_t* topk_idx, float* topk_gate, int32_t* counts, void* ws, size_t ws_bytes,
                           void* stream) {
+  NvtxScope range("moe_route_hash");
   MOE_TRY(check_common(cfg, ws, ws_bytes));
   if (cfg->n_tokens > 0 && (!h || !norm_w || !xn || !topk_idx || !topk_gate)) return MOE_ERR_INVALID_ARG;
   if (!counts) return MOE_ERR_INVALID_ARG;
@@ -246,6 +248,7 @@ moe_status moe_route_hash(const moe_config* cfg, const void* h, const void* norm
 moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const void* xn, int32_t* offsets,
                        int32_t* slot_row, int32_t* row_token, void* x_perm, void* ws, size_t ws_bytes,
                        void* stream) {
+  NvtxScope range("moe_permute");
   MOE_TRY(check_common(cfg, ws, ws_bytes));
   if (!offsets) return MOE_ERR_INVALID_ARG;
   if (cfg->n_tokens > 0 && (!topk_idx || !xn || !slot_row || !row_token || !x_perm)) return MOE_ERR_INVALID_ARG;
@@ -255,6 +258,7 @@ moe_status moe_permute(const moe_config* cfg, const int32_t* topk_idx, const voi
 moe_status moe_expert_ffn(const moe_config* cfg, int32_t n_groups, const int32_t* offsets, int32_t max_rows,
                           const void* x, const void* w_gate, const void* w_up, const void* w_down, int32_t d_ff,
                           void* y, void* ws, size_t ws_bytes, void* stream) {
+  NvtxScope range("moe_expert_ffn");
   MOE_TRY(check_common(cfg, ws, ws_bytes));
   if (n_groups < 1 || n_groups > 1024 || max_rows < 0 || d_ff < 1) return MOE_ERR_INVALID_ARG;
   if (offsets == nullptr && n_groups != 1) return MOE_ERR_INVALID_ARG;
@@ -266,6 +270,7 @@ moe_status moe_expert_ffn(const moe_config* cfg, int32_t n_groups, const int32_t
 
 moe_status moe_combine(const moe_config* cfg, const void* h, const void* y_perm, const int32_t* slot_row,
                        const float* topk_gate, const void* y_shared, void* out, void* stream) {
+  NvtxScope range("moe_combine");
   if (!config_ok(cfg)) return MOE_ERR_INVALID_ARG;
   if (!config_supported(cfg)) return MOE_ERR_UNSUPPORTED;
   if (cfg->n_tokens > 0 && (!h || !slot_row || !topk_gate || !out)) return MOE_ERR_INVALID_ARG;
@@ -299,14 +304,18 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const 
   void* x_perm = wsp(ws, L.x_perm);
   void* y_perm = wsp(ws, L.y_perm);
   void* y_shared = shared ? wsp(ws, L.y_shared) : nullptr;
-  auto mark = [&](void* ev) -> moe_status {
+  NvtxScope call_range("moe_layer_forward");
+  NvtxStages stages;
+  // records the trace event of a stage boundary and opens the next stage's range
+  auto mark = [&](void* ev, const char* next) -> moe_status {
+    stages.next(next);
     if (ev && cudaEventRecord((cudaEvent_t)ev, s) != cudaSuccess) return MOE_ERR_CUDA;
     return MOE_OK;
   };
-  MOE_TRY(mark(trace ? trace->start : nullptr));
+  MOE_TRY(mark(trace ? trace->start : nullptr, "route"));
   // the counts come from the permute's scan below
   MOE_TRY(route_impl(cfg, h, w->norm_w, w->w_router, bias, xn, scores, idx, gate, nullptr, ws, s));
-  MOE_TRY(mark(trace ? trace->routed : nullptr));
+  MOE_TRY(mark(trace ? trace->routed : nullptr, "permute"));
   const int R = (int)L.rows;
   const int N = cfg->n_tokens;
   void* act = wsp(ws, L.act);
@@ -317,55 +326,63 @@ moe_status moe_layer_forward(const moe_config* cfg, const moe_weights* w, const 
     MOE_TRY(launch_permute(idx, N, cfg->top_k, cfg->n_experts, (int)capacity_of(cfg), (int32_t*)wsp(ws, L.hist),
                            offsets, slot_row, row_token, s, offs_ext, N, counts));
     MOE_TRY(launch_gather(cfg->dtype, xn, slot_row, N, cfg->top_k, x_perm, cfg->d_model, s, hdr));
-    MOE_TRY(mark(trace ? trace->permuted : nullptr));
+    MOE_TRY(mark(trace ? trace->permuted : nullptr, "gate_up"));
     if (N > 0) {
       MOE_TRY(launch_gemm_tc(EPI_SWIGLU, x_perm, w->w_gate, w->w_up, offs_ext, cfg->n_experts + 1, R + N, cfg->d_ff,
                              cfg->d_model, act, cfg->d_ff, hdr, s, w->ws_gate, w->ws_up, xn, N));
-      MOE_TRY(mark(trace ? trace->gate_up : nullptr));
+      MOE_TRY(mark(trace ? trace->gate_up : nullptr, "down"));
       MOE_TRY(launch_gemm_tc(EPI_STORE, act, w->w_down, nullptr, offs_ext, cfg->n_experts + 1, R + N, cfg->d_model,
                              cfg->d_ff, y_perm, cfg->d_model, hdr, s, w->ws_down, nullptr));
     } else {
-      MOE_TRY(mark(trace ? trace->gate_up : nullptr));
+      MOE_TRY(mark(trace ? trace->gate_up : nullptr, "down"));
     }
-    MOE_TRY(mark(trace ? trace->down : nullptr));
-    MOE_TRY(mark(trace ? trace->shared : nullptr));  // included in the two launches above
+    MOE_TRY(mark(trace ? trace->down : nullptr, "shared"));
+    MOE_TRY(mark(trace ? trace->shared : nullptr, "combine"));  // included in the two launches above
     MOE_TRY(launch_combine(cfg->dtype, h, y_perm, slot_row, gate, nullptr, out, N, cfg->d_model, cfg->top_k, s,
                            offs_ext, cfg->n_experts));
-    MOE_TRY(mark(trace ? trace->combined : nullptr));
+    MOE_TRY(mark(trace ? trace->combined : nullptr, nullptr));
     return MOE_OK;
   }
   MOE_TRY(permute_impl(cfg, idx, xn, offsets, slot_row, row_token, x_perm, ws, s, counts));
-  MOE_TRY(mark(trace ? trace->permuted : nullptr));
+  MOE_TRY(mark(trace ? trace->permuted : nullptr, "gate_up"));
   if (R > 0) {
     if (use_tc(cfg)) {
       MOE_TRY(launch_gemm_tc(EPI_SWIGLU, x_perm, w->w_gate, w->w_up, offsets, cfg->n_experts, R, cfg->d_ff,
                              cfg->d_model, act, cfg->d_ff, hdr, s));
-      MOE_TRY(mark(trace ? trace->gate_up : nullptr));
+      MOE_TRY(mark(trace ? trace->gate_up : nullptr, "down"));
       MOE_TRY(launch_gemm_tc(EPI_STORE, act, w->w_down, nullptr, offsets, cfg->n_experts, R, cfg->d_model,
                              cfg->d_ff, y_perm, cfg->d_model, hdr, s));
     } else {
       MOE_TRY(launch_gemm_simt(cfg->dtype, EPI_SWIGLU, x_perm, w->w_gate, w->w_up, offsets, cfg->n_experts, R,
                                cfg->d_ff, cfg->d_model, act, cfg->d_ff, s));
-      MOE_TRY(mark(trace ? trace->gate_up : nullptr));
+      MOE_TRY(mark(trace ? trace->gate_up : nullptr, "down"));
       MOE_TRY(launch_gemm_simt(cfg->dtype, EPI_STORE, act, w->w_down, nullptr, offsets, cfg->n_experts, R,
                                cfg->d_model, cfg->d_ff, y_perm, cfg->d_model, s));
     }
   } else {
-    MOE_TRY(mark(trace ? trace->gate_up : nullptr));
+    MOE_TRY(mark(trace ? trace->gate_up : nullptr, "down"));
   }
-  MOE_TRY(mark(trace ? trace->down : nullptr));
+  MOE_TRY(mark(trace ? trace->down : nullptr, "shared"));
   if (shared && N > 0)
     MOE_TRY(ffn_impl(cfg, 1, nullptr, N, xn, w->ws_gate, w->ws_up, w->ws_down, cfg->d_ff_shared, y_shared, ws, s));
-  MOE_TRY(mark(trace ? trace->shared : nullptr));
+  MOE_TRY(mark(trace ? trace->shared : nullptr, "combine"));
   MOE_TRY(launch_combine(cfg->dtype, h, y_perm, slot_row, gate, y_shared, out, N, cfg->d_model, cfg->top_k, s));
-  MOE_TRY(mark(trace ? trace->combined : nullptr));
+  MOE_TRY(mark(trace ? trace->combined : nullptr, nullptr));
   return MOE_OK;
 }
 
 moe_status moe_bias_update(int32_t n_experts, const int32_t* counts, float target, float gamma, float* bias,
                            void* stream) {
+  NvtxScope range("moe_bias_update");
   if (n_experts < 1 || n_experts > 1024 || !counts || !bias) return MOE_ERR_INVALID_ARG;
   return launch_bias_update(n_experts, counts, target, gamma, bias, (cudaStream_t)stream);
+}
+
+moe_status moe_compute_load_stats(const moe_config* cfg, const int32_t* counts, const int32_t* offsets,
+                                  moe_load_stats* stats, void* stream) {
+  NvtxScope range("moe_compute_load_stats");
+  if (!config_ok(cfg) || !counts || !offsets || !stats) return MOE_ERR_INVALID_ARG;
+  return launch_load_stats(cfg->n_tokens * cfg->top_k, cfg->n_experts, counts, offsets, stats, (cudaStream_t)stream);
 }
 
 moe_status moe_check_device_error(void* ws, size_t ws_bytes, void* stream, int32_t* info) {

@@ -4,11 +4,33 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include "../../include/moe.h"
 
 namespace moe_host {
+
+// NVTX ranges on the host thread that enqueues the launches: one per entry
+// point and, inside moe_layer_forward, one per stage, so that a profiler
+// collecting NVTX attributes each kernel launch to its step.  Without such a
+// tool attached every NVTX call returns at once.
+struct NvtxScope {
+  explicit NvtxScope(const char* name) { nvtxRangePushA(name); }
+  ~NvtxScope() { nvtxRangePop(); }
+  NvtxScope(const NvtxScope&) = delete;
+  NvtxScope& operator=(const NvtxScope&) = delete;
+};
+
+struct NvtxStages {
+  bool open = false;
+  void next(const char* stage) {
+    if (open) nvtxRangePop();
+    open = stage != nullptr;
+    if (open) nvtxRangePushA(stage);
+  }
+  ~NvtxStages() { next(nullptr); }
+};
 
 // Config checks and the capacity rule shared by the entry points (moe_api.cu).
 bool config_ok(const moe_config* c);          // sizes and dtype valid
@@ -60,6 +82,10 @@ moe_status launch_combine(int dtype, const void* h, const void* y_perm, const in
 // a10: bias[e] += gamma * sign(target - counts[e]).
 moe_status launch_bias_update(int e, const int32_t* counts, float target, float gamma, float* bias,
                               cudaStream_t s);
+
+// a4 / a10: load statistics of one routing of `slots` = N*k slots (one block).
+moe_status launch_load_stats(int slots, int e, const int32_t* counts, const int32_t* offsets, moe_load_stats* stats,
+                             cudaStream_t s);
 
 // Grouped GEMM epilogues.
 enum GemmEpilogue { EPI_F32 = 0, EPI_SWIGLU = 1, EPI_STORE = 2 };

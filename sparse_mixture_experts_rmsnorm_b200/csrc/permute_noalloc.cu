@@ -69,6 +69,7 @@ extern "C" moe_status moe_permute_noalloc(const moe_config* cfg, const int32_t* 
                                           int32_t* offsets, int32_t* slot_row, int32_t* row_token, void* x_perm,
                                           void* stream) {
   using namespace moe_host;
+  NvtxScope range("moe_permute_noalloc");
   if (!config_ok(cfg)) return MOE_ERR_INVALID_ARG;
   if (!config_supported(cfg)) return MOE_ERR_UNSUPPORTED;
   if (!offsets) return MOE_ERR_INVALID_ARG;

@@ -97,6 +97,10 @@ def test_host_validation_before_any_launch():
     st = lib.moe_expert_ffn(ctypes.byref(good), 1, None, 100000, 256, 256, 256, 256, 128, 256, 256, 1 << 30, None)
     assert st == moe.MOE_ERR_WORKSPACE
     assert lib.moe_bias_update(0, 256, 1.0, 1e-3, 256, None) == moe.MOE_ERR_INVALID_ARG
+    # load statistics: a NULL buffer or a bad config
+    assert lib.moe_compute_load_stats(ctypes.byref(good), 256, None, 256, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_compute_load_stats(ctypes.byref(bad), 256, 256, 256, None) == moe.MOE_ERR_INVALID_ARG
+    assert ctypes.sizeof(moe.MoeLoadStats) == 20
     # combine: the expert rows are required while any slot can be kept
     st = lib.moe_combine(ctypes.byref(good), 256, None, 256, 256, None, 256, None)
     assert st == moe.MOE_ERR_INVALID_ARG

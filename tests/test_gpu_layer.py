@@ -321,6 +321,40 @@ def test_bias_update_bit_exact(torch_cuda):
     assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
 
 
+# ----------------------------------------------------------------- load statistics
+
+@pytest.mark.parametrize("capacity_factor", [0.0, 1.0])
+def test_load_stats_match_oracle(torch_cuda, capacity_factor):
+    torch = torch_cuda
+    import ctypes
+    import sparse_mixture_experts_rmsnorm_b200 as moe
+    cfg = mi.LayerConfig(name="stats", n_tokens=1000, d_model=256, n_experts=16, top_k=4, d_ff=64,
+                         capacity_factor=capacity_factor, router_sigma=0.1, seed=5)
+    E = cfg.n_experts
+    g = run_gpu_layer(cfg, with_route=False)
+    # the expected statistics come from the oracle's counts and permutation of
+    # the GPU's chosen experts (the routing itself is compared elsewhere)
+    idx = g["topk_idx"]
+    offsets, _, _ = oracle.permute(idx, E, capacity(cfg))
+    ref = oracle.load_stats(oracle.expert_counts(idx, E), offsets, cfg.n_tokens, cfg.top_k, E)
+    stats = torch.zeros(ctypes.sizeof(moe.MoeLoadStats), dtype=torch.uint8, device="cuda")
+    moe.moe_compute_load_stats(lib_config(cfg), torch.tensor(g["counts"], device="cuda"),
+                               torch.tensor(g["offsets"], device="cuda"), stats)
+    got = moe.MoeLoadStats.from_buffer_copy(bytes(stats.cpu().numpy()))
+    assert (got.routed, got.kept, got.dropped, got.max_count) == (ref["routed"], ref["kept"], ref["dropped"],
+                                                                  ref["max_count"])
+    assert np.float32(got.max_over_mean).view(np.uint32) == ref["max_over_mean"].view(np.uint32)
+    assert (got.dropped > 0) == (capacity_factor > 0)
+
+    # no tokens: every field zero
+    empty = cfg.with_(n_tokens=0)
+    z = torch.zeros(E + 1, dtype=torch.int32, device="cuda")
+    stats.fill_(0xFF)
+    moe.moe_compute_load_stats(lib_config(empty), z, z, stats)
+    got = moe.MoeLoadStats.from_buffer_copy(bytes(stats.cpu().numpy()))
+    assert (got.routed, got.kept, got.dropped, got.max_count, got.max_over_mean) == (0, 0, 0, 0, 0.0)
+
+
 # ----------------------------------------------------------------- bounded device wait
 
 def test_device_wait_times_out_and_reports(torch_cuda):

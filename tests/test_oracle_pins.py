@@ -184,6 +184,39 @@ def test_glossary_example_with_capacity_two():
     assert dropped == [4 * 2 + 0, 5 * 2 + 1]  # token 4 -> expert 6, token 5 -> expert 3
 
 
+def test_load_stats_of_the_glossary_example():
+    # The printed example: 12 slots over 8 experts (mean load 1.5), the
+    # busiest experts (3 and 6) take three tokens each, so max/mean = 2; a
+    # capacity of 2 drops one slot at each of them and at no other expert.
+    fx = json.load(open(os.path.join(GOLDEN, "glossary_top2_example.json")))
+    idx = np.array(fx["experts_per_token"])
+    n, E, k = fx["n_tokens"], fx["n_experts"], fx["top_k"]
+    counts = np.array(fx["tokens_per_expert"])
+    free, _, _ = oracle.permute(idx, E)
+    st = oracle.load_stats(counts, free, n, k, E)
+    assert (st["routed"], st["kept"], st["dropped"], st["max_count"]) == (12, 12, 0, 3)
+    assert st["max_over_mean"] == np.float32(2.0)
+    capped, _, _ = oracle.permute(idx, E, capacity=2)
+    st = oracle.load_stats(counts, capped, n, k, E)
+    # the maximum is taken before the cut, as the bias update's usage is
+    assert (st["routed"], st["kept"], st["dropped"], st["max_count"]) == (12, 10, 2, 3)
+    assert st["max_over_mean"] == np.float32(2.0)
+
+
+def test_load_stats_closed_forms():
+    # perfect balance gives max/mean = 1 exactly; every slot on one expert gives E
+    E, k, n = 16, 4, 64
+    even = np.full(E, n * k // E)
+    st = oracle.load_stats(even, np.concatenate([[0], np.cumsum(even)]), n, k, E)
+    assert st["max_over_mean"] == np.float32(1.0) and st["dropped"] == 0
+    one = np.zeros(E, dtype=np.int64)
+    one[7] = n * k
+    st = oracle.load_stats(one, np.concatenate([[0], np.cumsum(one)]), n, k, E)
+    assert st["max_over_mean"] == np.float32(E) and st["max_count"] == n * k
+    st = oracle.load_stats(np.zeros(E), np.zeros(E + 1), 0, k, E)
+    assert (st["routed"], st["kept"], st["dropped"], st["max_count"], st["max_over_mean"]) == (0, 0, 0, 0, 0.0)
+
+
 def test_permute_brute_force_small():
     for _ in range(30):
         n, E, k = 13, 5, 2
