@@ -25,3 +25,16 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(scope="module")
+def torch_cuda():
+    """torch with a CUDA device, the library loaded (it fails loudly when its
+    build is missing) and the device input generator built."""
+    import torch
+    assert torch.cuda.is_available()
+    import moe_inputs as mi
+    import sparse_mixture_experts_rmsnorm_b200  # noqa: F401
+    if not os.path.exists(mi.CUDA_LIB):
+        mi.build(cuda=True)
+    return torch

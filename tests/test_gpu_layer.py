@@ -22,16 +22,6 @@ pytestmark = pytest.mark.gpu
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
 
-@pytest.fixture(scope="module")
-def torch_cuda():
-    import torch
-    assert torch.cuda.is_available()
-    import sparse_mixture_experts_rmsnorm_b200  # noqa: F401  (fails loudly when the library is missing)
-    if not os.path.exists(mi.CUDA_LIB):
-        mi.build(cuda=True)
-    return torch
-
-
 def _full_oracle(cfg):
     a = {n: mi.host_tensor(cfg, n) for n in mi.layer_tensor_specs(cfg)}
     return oracle.layer_forward(a["h"], a["norm_w"], a["w_router"], a["bias"], a["w_gate"], a["w_up"],
