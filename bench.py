@@ -16,6 +16,10 @@ Under torchrun every rank runs an independent replica of the layer on its
 own GPU (the layer shards by tokens and needs no exchange); the time is the
 max over ranks and the value counts the tokens of all ranks.
 
+The line also carries the routing's load statistics ("load": routed, kept
+and dropped slots, the largest expert count, max/mean load), taken from the
+library outside the timed region.
+
 --impl reference times the CPU oracle (plain float64 numpy) on a bounded
 sample of the same workload on the host cores; rank 0 alone runs it.
 
