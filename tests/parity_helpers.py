@@ -11,11 +11,11 @@ import numpy as np
 import moe_inputs as mi
 import oracle
 
-# Routing comparisons skip tokens whose oracle keys are this close.  Two keys
-# further apart cannot swap while each fp32 key is within KEY_TIE / 2 of the
-# oracle's, which test_gpu_configs checks on every workload (largest errors
+# Routing comparisons skip tokens whose oracle keys are this close: the
+# tolerance stated for this layer.  test_gpu_configs also checks that every
+# fp32 key lies within KEY_TIE of the oracle's on each workload (largest errors
 # measured on B200: 6.6e-7 for the tensor-core router, 8.9e-7 on the CUDA cores).
-KEY_TIE = 2e-6
+KEY_TIE = 1e-6
 BF16_REL_RMS = 2e-2     # bf16 layers: max |gpu - oracle| / rms(oracle)
 F32_MAX_ABS = 1e-4      # fp32 layer: max |gpu - oracle|
 

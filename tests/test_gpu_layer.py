@@ -2,7 +2,7 @@
 
 Every test here needs a B200 (sm_100a).  Routing, counts, permutation and
 drop masks are compared bit-exactly (tokens whose oracle selection keys are
-within KEY_TIE = 2e-6 of each other are skipped); outputs within max-abs 1e-4 (fp32
+within KEY_TIE = 1e-6 of each other are skipped); outputs within max-abs 1e-4 (fp32
 layer) or 2e-2 of the output RMS (bf16 layers, fp32 accumulation); bias
 updates bit-exactly.
 """
@@ -288,9 +288,7 @@ def test_router_tc_routing_bit_exact(torch_cuda, E, k):
     np.testing.assert_array_equal(g["xn"], ref["xn"])
     np.testing.assert_allclose(g["scores"], ref["scores"], rtol=2e-5, atol=1e-9)
     skipped = check_routing(g, ref, k)
-    # a property of the inputs alone (7 and 16 of the 777 tokens have top keys within KEY_TIE): the
-    # comparison must still cover most tokens
-    assert skipped < 0.05 * cfg.n_tokens
+    assert skipped < 0.02 * cfg.n_tokens
     check_permutation(g, E, -1)
 
 
