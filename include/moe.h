@@ -307,8 +307,9 @@ moe_status moe_set_wait_timeout_ns(int64_t ns);
  * sizes), 1 = single-SM tiles, 2 = SM-pair tiles, 3 = swapped-operand SM-pair
  * tiles for both expert GEMMs where the shape allows (K % 64 == 0).  The
  * tensor-core router (bf16, E >= 64, N >= 512) always runs single-SM
- * 128 x 128 tiles whose fp32 accumulation restarts every 256 along d, the
- * partial sums added in fp32 registers, whatever the mode.  Results are the
+ * tiles of 128 rows and 128 columns (256 when that takes fewer waves) whose
+ * fp32 accumulation restarts every 256 along d, the partial sums added in
+ * fp32 registers, whatever the mode.  Results are the
  * same up to floating-point summation order; this is a performance control.
  * MOE_ERR_INVALID_ARG for any other mode. */
 moe_status moe_set_gemm_tiling(int32_t mode);

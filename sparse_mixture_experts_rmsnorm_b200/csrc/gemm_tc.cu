@@ -27,19 +27,21 @@
 // every tile of a decode step) runs as M = 64 MMAs; its accumulator keeps row
 // r in TMEM lane (r / 16) * 32 + r % 16, the first 16 lanes of each quarter.
 // For SwiGLU, B holds 128 gate rows then 128 up rows of the same hidden
-// units, so one N = 256 MMA produces both halves.  A plain-epilogue launch
-// with too few tiles to fill the SMs (the router's logits) uses 128-column
-// tiles: one B box per stage and N = 128 MMAs.
-// The fp32 epilogue (router logits) always runs 128-column tiles and
-// accumulates in K-chunks.  The tensor cores' fp32 accumulator loses more
+// units, so one N = 256 MMA produces both halves.  A plain-store launch with
+// too few tiles to fill the SMs uses 128-column tiles: one B box per stage
+// and N = 128 MMAs.
+// The fp32 epilogue (router logits) runs 128-column tiles (256-column ones
+// when those take fewer waves) and accumulates in K-chunks.  The tensor cores' fp32 accumulator loses more
 // per step than a round-to-nearest add: measured on B200 against a float64
 // router with K = 7168 and 256 experts, one accumulator per tile put the
 // selection keys (softmax score + bias) off by up to 1.2e-5, enough to swap
 // two experts whose keys differ by 1.1e-6; chunks of 256 (or 128) along K
 // bring that to 6.6e-7, and chunks of 512 to 8.9e-7.  So each chunk of
 // TC_F32_CHUNK_KB k-blocks starts a fresh accumulator in one of four
-// 128-column TMEM slots, and the epilogue warps add the chunks in order in
-// fp32 registers (round-to-nearest) before the single store of the row.
+// 128-column (or two 256-column) TMEM slots, and eight epilogue warps, two
+// per TMEM lane quarter and each with half the columns, add the chunks in
+// order in fp32 registers (round-to-nearest) before the single store of the
+// row.
 // Tiles are numbered group-major, then n-tile, then m-tile, so CTAs working
 // at the same time share weight tiles through L2.
 // Every mbarrier wait is bounded: on time-out the block records
@@ -62,14 +64,32 @@ constexpr int TC_STAGE_BYTES = TC_A_BYTES + 2 * TC_B_HALF_BYTES;
 constexpr int TC_EPI_STAGE_BYTES = 32 * 128;  // one warp's 32 x 64 bf16 output block (TMA-store epilogue)
 constexpr int TC_SMEM_BYTES = TC_STAGES * TC_STAGE_BYTES + 4 * TC_EPI_STAGE_BYTES + 1024;  // + alignment slack
 constexpr int TC_THREADS = 192;
+// The fp32 epilogue runs eight epilogue warps, two per TMEM lane quarter,
+// each summing half of a tile's columns, so that a 256-column tile keeps at
+// most 128 partial sums per thread.
+template <int EPI>
+constexpr int tc_threads() {
+  return EPI == moe_host::EPI_F32 ? 320 : TC_THREADS;
+}
 constexpr int TC_F32_CHUNK_KB = 4;  // k-blocks (of 64) per fp32 partial accumulator: K = 256
 
-// Writes one fp32 row of 128 columns n0 .. n0 + 127, masked to columns < nout.
-__device__ __forceinline__ void store_row128_f32(const TcArgs& args, int row, int n0, const float (&v)[128]) {
+// tcgen05.ld of 16 columns of the warp's 32 TMEM lanes (16 registers a thread).
+#define MOE_TMEM_LD16(taddr, r)                                                                                   \
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, " \
+               "%13, %14, %15}, [%16];"                                                                         \
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),  \
+                 "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),         \
+                 "=r"(r[15])                                                                                      \
+               : "r"(taddr))
+
+// Writes `ncols` (a multiple of 4, at most 128) fp32 values of one row from
+// column n0 on, masked to columns < nout.
+__device__ __forceinline__ void store_row_f32(const TcArgs& args, int row, int n0, int ncols, const float (&v)[128]) {
   float* out = reinterpret_cast<float*>(args.C) + (size_t)row * args.ldc;
   const bool vec = (args.ldc & 3) == 0 && (reinterpret_cast<uintptr_t>(args.C) & 15) == 0;
 #pragma unroll
   for (int c = 0; c < 128; c += 4) {
+    if (c >= ncols) break;
     const int col = n0 + c;
     if (vec && col + 4 <= args.nout) {
       *reinterpret_cast<float4*>(out + col) = make_float4(v[c], v[c + 1], v[c + 2], v[c + 3]);
@@ -82,7 +102,7 @@ __device__ __forceinline__ void store_row128_f32(const TcArgs& args, int row, in
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(tc_threads<EPI>(), 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                    const __grid_constant__ CUtensorMap map_b2, const __grid_constant__ CUtensorMap map_sb,
                    const __grid_constant__ CUtensorMap map_sb2, const __grid_constant__ CUtensorMap map_sa,
@@ -90,11 +110,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[TC_STAGES];
   __shared__ __align__(8) uint64_t empty_bar[TC_STAGES];
-  // accumulator slots: two of 256 columns (one per tile), or four of 128
-  // columns (one per K-chunk) for the fp32 epilogue
+  // accumulator slots: two of 256 columns (one per tile); for the fp32
+  // epilogue one per K-chunk, four of 128 columns (128-column tiles) or two
+  // of 256 (256-column tiles)
   constexpr bool F32 = EPI == moe_host::EPI_F32;
   constexpr int NBUF = F32 ? 4 : 2;
-  constexpr uint32_t SLOT_COLS = F32 ? 128u : (uint32_t)TC_BN;
   __shared__ __align__(8) uint64_t tfull_bar[NBUF];
   __shared__ __align__(8) uint64_t tempty_bar[NBUF];
   __shared__ __align__(8) uint64_t drain_bar;
@@ -130,7 +150,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     }
     for (int b = 0; b < NBUF; ++b) {
       mbar_init(&tfull_bar[b], 1);
-      mbar_init(&tempty_bar[b], 4);
+      mbar_init(&tempty_bar[b], F32 ? 8 : 4);  // one arrival per epilogue warp
     }
     mbar_init(&drain_bar, 1);
     fence_barrier_init();
@@ -147,6 +167,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const uint32_t tmem_base = tmem_base_sh;
   const int total_tiles = prefix_sh[G];
   const int nk = (args.K + TC_BK - 1) / TC_BK;
+  const uint32_t slot_cols = (F32 && args.narrow) ? 128u : (uint32_t)TC_BN;
+  const int nbuf = (F32 && args.narrow) ? 4 : 2;
   // k-blocks per accumulator and accumulators per tile
   const int chunk_kb = F32 ? TC_F32_CHUNK_KB : nk;
   const int n_chunks = F32 ? (nk + TC_F32_CHUNK_KB - 1) / TC_F32_CHUNK_KB : 1;
@@ -232,7 +254,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t d_tmem = tmem_base + (uint32_t)buf * SLOT_COLS;
+          const uint32_t d_tmem = tmem_base + (uint32_t)buf * slot_cols;
           const int kb0 = c * chunk_kb;
           const int kb1 = kb0 + chunk_kb < nk ? kb0 + chunk_kb : nk;
           for (int kb = kb0; kb < kb1; ++kb) {
@@ -256,7 +278,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
           if (!ok) break;
           tc_commit(&tfull_bar[buf]);
-          if (++buf == NBUF) {
+          if (++buf == nbuf) {
             buf = 0;
             bphase ^= 1u;
           }
@@ -267,7 +289,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_wait_bounded(&drain_bar, 0, args.wait_ns, nullptr, args.hdr, KID_GEMM_TC, SITE_DRAIN);
     }
   } else {
-    // ======================= epilogue (warps 2..5) =======================
+    // ============ epilogue (warps 2..5; for the fp32 epilogue 2..9) ============
     const int quarter = warp & 3;  // TMEM lanes this warp may access
     const int r_local = quarter * 32 + lane;
     int buf = 0;
@@ -278,6 +300,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // the tile's K-chunks, summed in order in fp32 registers
         const bool half = tl.row_end - tl.row0 <= 64;
         const int row = half ? tl.row0 + quarter * 16 + (lane & 15) : tl.row0 + r_local;
+        // warps 2..5 take the first half of the tile's columns, warps 6..9 the second
+        const int my_cols = (int)slot_cols / 2;  // 64 or 128
+        const int col0 = ((warp - 2) >> 2) * my_cols;
         float acc[128];
 #pragma unroll
         for (int i = 0; i < 128; ++i) acc[i] = 0.0f;
@@ -289,25 +314,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           ok = __shfl_sync(0xffffffffu, ok, 0);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t tb = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)buf * SLOT_COLS;
+          const uint32_t tb =
+              tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)buf * slot_cols + (uint32_t)col0;
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            uint32_t a[32];
-            MOE_TMEM_LD32(tb + 32 * j, a);
+          for (int j = 0; j < 8; ++j) {  // 16 columns at a time, so the sums and a load fit the registers
+            if (16 * j >= my_cols) break;
+            uint32_t a[16];
+            MOE_TMEM_LD16(tb + 16 * j, a);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc[32 * j + i] = __fadd_rn(acc[32 * j + i], __uint_as_float(a[i]));
+            for (int i = 0; i < 16; ++i) acc[16 * j + i] = __fadd_rn(acc[16 * j + i], __uint_as_float(a[i]));
           }
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty_bar[buf]);
-          if (++buf == NBUF) {
+          if (++buf == nbuf) {
             buf = 0;
             bphase ^= 1u;
           }
         }
         if (!ok) break;
-        if (row < tl.row_end && (!half || lane < 16)) store_row128_f32(args, row, tl.n0, acc);
+        if (row < tl.row_end && (!half || lane < 16)) store_row_f32(args, row, tl.n0 + col0, my_cols, acc);
         continue;
       }
       bool ok = true;
@@ -317,7 +344,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)buf * SLOT_COLS;
+      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)buf * slot_cols;
       // M = 64 accumulators keep row r in lane (r / 16) * 32 + r % 16: lanes
       // 0..15 of each warp's quarter
       const bool half = tl.row_end - tl.row0 <= 64;
@@ -333,7 +360,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty_bar[buf]);
-      if (++buf == NBUF) {
+      if (++buf == nbuf) {
         buf = 0;
         bphase ^= 1u;
       }
@@ -416,7 +443,8 @@ static moe_status launch_tc_t(const CUtensorMap& ma, const CUtensorMap& mb, cons
   static SmemLimit lim;
   const moe_status st = ensure_smem_limit(moe::gemm_tc_kernel<EPI>, moe::TC_SMEM_BYTES, lim);
   if (st != MOE_OK) return st;
-  moe::gemm_tc_kernel<EPI><<<grid, moe::TC_THREADS, moe::TC_SMEM_BYTES, s>>>(ma, mb, mb2, msb, msb2, msa, mc, args);
+  moe::gemm_tc_kernel<EPI><<<grid, moe::tc_threads<EPI>(), moe::TC_SMEM_BYTES, s>>>(ma, mb, mb2, msb, msb2, msa, mc,
+                                                                                    args);
   return launch_status();
 }
 
@@ -513,14 +541,20 @@ moe_status launch_gemm_tc(int epi, const void* a, const void* b, const void* b2,
   // Upper bound on the number of tiles; the exact count lives on the device.
   const int64_t m_tiles = (int64_t)(max_rows + moe::TC_BM - 1) / moe::TC_BM + (offsets ? groups : 0);
   if (epi == EPI_F32) {
-    // fp32 outputs (the router's logits) always take single-SM 128-column
-    // tiles, accumulated in K-chunks, whatever the tiling setting
-    args.narrow = 1;
-    args.out_cols = 128;
-    args.n_tiles = (nout + 127) / 128;
+    // fp32 outputs (the router's logits) take single-SM tiles accumulated in
+    // K-chunks, whatever the tiling setting: 128 columns wide, or 256 when
+    // that takes fewer waves.  A 256-column tile loads 1.5 times the bytes of
+    // a 128-column one per k-block (A once, B twice), and the router's loads
+    // set its pace, so it counts as 1.5 narrow tiles.
+    const int64_t sms = sm_count();
+    const int64_t narrow_waves = (m_tiles * ((nout + 127) / 128) + sms - 1) / sms;
+    const int64_t wide_waves = (m_tiles * ((nout + 255) / 256) + sms - 1) / sms;
+    const bool wide = 3 * wide_waves < 2 * narrow_waves;
+    args.narrow = wide ? 0 : 1;
+    args.out_cols = wide ? 256 : 128;
+    args.n_tiles = (nout + args.out_cols - 1) / args.out_cols;
     const int64_t tiles = m_tiles * args.n_tiles;
-    return launch_tc_t<EPI_F32>(ma, mb, mb2, msb, msb2, msa, mc, args, (int)(tiles < sm_count() ? tiles : sm_count()),
-                                s);
+    return launch_tc_t<EPI_F32>(ma, mb, mb2, msb, msb2, msa, mc, args, (int)(tiles < sms ? tiles : sms), s);
   }
   const int mode = forced == 3 ? 0 : forced;
   // A plain-store launch that would leave more than half the SMs idle runs

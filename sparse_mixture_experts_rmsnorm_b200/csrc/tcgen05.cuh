@@ -347,8 +347,8 @@ int64_t tc2_pairs_launched(int epi, int64_t max_rows, int groups_bound, int n_ti
 //    sizes, pairs_picked);
 // 1: single-SM tiles only; 2: SM-pair tiles only; 3: the swapped-operand
 //    kernel for the expert GEMMs it supports (the rest take 0's choice).
-// The fp32 logits (the router) always take single-SM 128-column tiles with
-// K-chunked accumulation, whatever the mode.
+// The fp32 logits (the router) always take single-SM tiles (128 or 256
+// columns) with K-chunked accumulation, whatever the mode.
 void set_tc_pairing(int mode);
 int tc_pairing();
 }  // namespace moe_host

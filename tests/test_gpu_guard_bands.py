@@ -6,8 +6,8 @@ a known byte inside one larger allocation.  After the layer forward and the
 staged calls, every band byte must be unchanged.  The workloads reach each
 kernel path: the CUDA-core fp32 GEMMs, the swapped-operand and single-SM
 tcgen05 GEMMs, the folded and the separate shared expert, the tensor-core
-router, capacity drops, the bulk-copy and the column-split row scatter, and
-d_model and d_ff that are not multiples of 64.  Parity of the values is
+router (128- and 256-column tiles), capacity drops, the bulk-copy and the
+column-split row scatter, and d_model and d_ff that are not multiples of 64.  Parity of the values is
 checked by the other GPU tests.
 """
 import numpy as np
@@ -35,6 +35,8 @@ CASES = {
                        bias=("uniform", -0.01, 0.01), seed=6),
     "bf16 tensor-core router":
         mi.LayerConfig(name="g4", n_tokens=600, d_model=256, n_experts=128, top_k=4, d_ff=64, seed=7),
+    "bf16 tensor-core router, 256-column tiles":
+        mi.LayerConfig(name="g6", n_tokens=16384, d_model=256, n_experts=256, top_k=8, d_ff=64, seed=9),
     "bf16 d_model and d_ff not multiples of 64":
         mi.LayerConfig(name="g5", n_tokens=400, d_model=200, n_experts=8, top_k=2, d_ff=136, d_ff_shared=72,
                        capacity_factor=1.1, seed=8),

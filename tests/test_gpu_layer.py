@@ -279,9 +279,11 @@ def test_folded_shared_expert_many_groups(torch_cuda, gemm_tiling, mode):
 
 # ----------------------------------------------------------------- router on the tensor cores
 
-@pytest.mark.parametrize("E,k", [(64, 6), (256, 8)])
-def test_router_tc_routing_bit_exact(torch_cuda, E, k):
-    cfg = mi.LayerConfig(name="router", n_tokens=777, d_model=1024, n_experts=E, top_k=k, d_ff=64,
+# 777 tokens run 128-column router tiles; 16424 tokens with 256 experts run
+# 256-column ones (fewer waves), the last of 129 row tiles 40 rows (M = 64)
+@pytest.mark.parametrize("E,k,N", [(64, 6, 777), (256, 8, 777), (256, 8, 16424)])
+def test_router_tc_routing_bit_exact(torch_cuda, E, k, N):
+    cfg = mi.LayerConfig(name="router", n_tokens=N, d_model=1024, n_experts=E, top_k=k, d_ff=64,
                          bias=("uniform", -0.01, 0.01), seed=3)
     g = run_gpu_layer(cfg)
     ref = oracle_routing(cfg)
